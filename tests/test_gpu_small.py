@@ -1,0 +1,271 @@
+"""GPU parity on the small workloads: the CUDA path (through the C ABI) against
+the CPU oracle, element by element and byte by byte.
+
+Covers: encoder bitstream identity (payload bytes and grouped offsets),
+decode+reduce on oracle-encoded and GPU-encoded residents, block_stride k,
+delta chains, uint64 promotion, invalid pixels, block decode, malformed
+streams and delta invalidation, deferred (wait=False) status.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import virtual_imaging_b200 as V
+import workloads as W
+from qem_testlib import export_all, gpu_encode, image, oracle_resident, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["c1", "c2", "s17", "s19", "s257"]
+
+
+@pytest.fixture(scope="module")
+def data():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            w = W.workload(name)
+            x = w.host_counts()
+            cache[name] = (w, x, O.encode(x, w.dtype_bits))
+        return cache[name]
+
+    return get
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_encoder_bitstream_identical(data, name):
+    w, x, enc = data(name)
+    res = gpu_encode(w, x)
+    for b, (g, p) in enumerate(export_all(res, w.n_blocks)):
+        assert (g == enc.groups[b]).all(), (name, b)
+        assert p.size == enc.payloads[b].size and (p == enc.payloads[b]).all(), (name, b)
+    info = res.info()
+    assert info["payload_bytes"] == enc.payload_bytes()
+    assert sum(info["form_count"].values()) == w.n_blocks * w.n_pixels
+    res.free()
+
+
+@pytest.mark.parametrize("name", SMALL)
+@pytest.mark.parametrize("source", ["oracle", "gpu"])
+def test_masked_sum_matches(data, name, source):
+    w, x, enc = data(name)
+    res = oracle_resident(w, enc) if source == "oracle" else gpu_encode(w, x)
+    for k in (1, 2, 3):
+        for mname, m in w.masks.items():
+            want = O.dense_masked_sum(x, m, None, k)
+            got = image(res, m, k)
+            assert got.shape == (math.ceil(w.n_blocks / k), 512)
+            assert (got == want).all(), (name, mname, k)
+    # the full-detector image is all pixels
+    full = np.ones(w.n_pixels, np.uint8)
+    assert (image(res, full) == O.dense_masked_sum(x, full)).all()
+    res.free()
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_decode_blocks_roundtrip(data, name):
+    w, x, enc = data(name)
+    res = gpu_encode(w, x)
+    out = res.decode_blocks(0, w.n_blocks)
+    assert (out.cpu().numpy() == x).all()
+    if w.n_blocks > 1:
+        part = res.decode_blocks(w.n_blocks - 1, 1)
+        assert (part.cpu().numpy() == x[-512:]).all()
+    res.free()
+
+
+def test_delta_chain_c2(data):
+    w, x, enc = data("c2")
+    res = gpu_encode(w, x)
+    for k in (1, 3):
+        img = image(res, w.drag[0], k)
+        assert (img == O.dense_masked_sum(x, w.drag[0], None, k)).all()
+        for t in range(1, len(w.drag)):
+            img = image(res, w.drag[t], k, delta=True)
+            assert (img == O.dense_masked_sum(x, w.drag[t], None, k)).all(), (k, t)
+    res.free()
+
+
+def test_invalid_pixels(data):
+    w, x, enc = data("s19")
+    valid = W.invalid_mask(w, 3)
+    res = gpu_encode(w, x, valid)
+    for mname, m in w.masks.items():
+        assert (image(res, m, 1) == O.dense_masked_sum(x, m, valid, 1)).all(), mname
+    frames = res.decode_blocks(0, w.n_blocks).cpu().numpy()
+    assert (frames == O.dense_decode_blocks(x, 0, w.n_blocks, valid)).all()
+    assert res.info()["n_valid"] == w.n_pixels - 3
+    res.free()
+
+
+def test_uint64_promotion_257():
+    """Page "Contract": uint64 when a full-detector sum could exceed 2**32."""
+    w = W.workload("s257")
+    P = w.n_pixels
+    x = np.full((512, P), 65535, np.uint16)
+    x[::7, ::3] = 65534
+    res = gpu_encode(w, x)
+    assert res.info()["out_bits_auto"] == 64
+    img = res.masked_sum(to_dev(np.ones(P, np.uint8)))
+    assert img.dtype == torch.int64
+    got = V.as_unsigned(img)[0]
+    closed = P * 65535 - np.array([len(range(0, P, 3)) if i % 7 == 0 else 0 for i in range(512)])
+    assert (got == closed.astype(np.uint64)).all()
+    assert int(got.max()) > 2 ** 32
+    with pytest.raises(V.QemError):
+        res.masked_sum(to_dev(np.ones(P, np.uint8)), out_bits=32)
+    res.free()
+
+
+def test_forced_uint64_and_auto_uint32(data):
+    w, x, enc = data("c2")
+    res = gpu_encode(w, x)
+    assert res.info()["out_bits_auto"] == 32
+    full = np.ones(w.n_pixels, np.uint8)
+    a = image(res, full, 1, out_bits=64)
+    b = image(res, full, 1)
+    assert (a == b).all() and (a == O.dense_masked_sum(x, full)).all()
+    res.free()
+
+
+def test_stride_counters(data):
+    w, x, enc = data("c2")
+    res = gpu_encode(w, x)
+    res.counters()
+    for k in (1, 2, 3, 5, 8, 9):
+        image(res, w.masks["bf"], k)
+        rows, streams = res.counters()
+        assert rows == math.ceil(w.n_blocks / k)
+        assert streams == rows * int(w.masks["bf"].sum())
+    res.free()
+
+
+def _corrupt_reserved(enc, b, p_idx):
+    g = enc.groups[b]
+    gi, j = divmod(p_idx, 32)
+    e = lambda j: int((g[gi, 1 + j // 2] >> (16 * (j & 1))) & 0xFFFF)
+    a = int(g[gi, 0]) + (e(j - 1) if j else 0)
+    pay = [p.copy() for p in enc.payloads]
+    pay[b][a + 1] |= 0x80
+    return pay
+
+
+def test_malformed_reserved_bit_and_taint(data):
+    w, x, enc = data("c2")
+    q = int(np.nonzero(w.masks["bf"])[0][5])
+    pay = _corrupt_reserved(enc, 1, q)
+    res = oracle_resident(w, enc, payloads=pay)
+    # the oracle agrees it is malformed
+    with pytest.raises(O.MalformedStream):
+        O.block_masked_sum(enc.groups[1], pay[1], 16, w.n_pixels, np.array([q]), np.array([1]))
+    # stride 2 touches blocks 0,2,4,6 only: no error
+    assert (image(res, w.masks["bf"], 2) == O.dense_masked_sum(x, w.masks["bf"], None, 2)).all()
+    # stride 1 touches block 1: the query raises and taints the stride-1 baseline
+    with pytest.raises(V.MalformedStream):
+        image(res, w.masks["bf"], 1)
+    with pytest.raises(V.TaintedBaseline):
+        image(res, w.masks["adf"], 1, delta=True)
+    # a full query with a mask that avoids the stream clears the taint
+    m = w.masks["adf"]
+    assert (image(res, m, 1) == O.dense_masked_sum(x, m, None, 1)).all()
+    d = image(res, w.masks["adf"] | (np.arange(w.n_pixels) == 0).astype(np.uint8), 1, delta=True)
+    assert (d == O.dense_masked_sum(x, w.masks["adf"] | (np.arange(w.n_pixels) == 0), None, 1)).all()
+    # block decode of the bad block raises too
+    with pytest.raises(V.MalformedStream):
+        res.decode_blocks(1, 1)
+    res.free()
+
+
+def test_malformed_shortened_extent(data):
+    """Page "Verification": a shortened stream extent is rejected."""
+    w, x, enc = data("s17")
+    for form in (1, 2, 3, 4):
+        for b in range(w.n_blocks):
+            g, pay = enc.groups[b], enc.payloads[b]
+            found = None
+            for q in range(w.n_pixels):
+                gi, j = divmod(q, 32)
+                e = lambda jj: int((g[gi, 1 + jj // 2] >> (16 * (jj & 1))) & 0xFFFF)
+                a = int(g[gi, 0]) + (e(j - 1) if j else 0)
+                if e(j) > (e(j - 1) if j else 0) and (pay[a] & 7) == form:
+                    found = (q, gi, j)
+                    break
+            if found:
+                break
+        if not found:
+            continue
+        q, gi, j = found
+        bad = [gg.copy() for gg in enc.groups]
+        bad[b][gi, 1 + j // 2] = np.uint32(int(bad[b][gi, 1 + j // 2]) - (1 << (16 * (j & 1))))
+        res = oracle_resident(w, enc, groups=bad)
+        m = np.zeros(w.n_pixels, np.uint8)
+        m[q] = 1
+        with pytest.raises(V.MalformedStream):
+            image(res, m, 1)
+        res.free()
+
+
+def test_malformed_flipped_bits_match_oracle(data):
+    """Every single-bit flip in a paired stream: GPU and oracle agree on error/no-error and value."""
+    w, x, enc = data("c1")
+    g, pay = enc.groups[0], enc.payloads[0]
+    bf = np.nonzero(w.masks["bf"])[0]
+    q = int(bf[3])
+    gi, j = divmod(q, 32)
+    e = lambda jj: int((g[gi, 1 + jj // 2] >> (16 * (jj & 1))) & 0xFFFF)
+    a, z = int(g[gi, 0]) + (e(j - 1) if j else 0), int(g[gi, 0]) + e(j)
+    assert pay[a] & 7 == 3
+    m = np.zeros(w.n_pixels, np.uint8)
+    m[q] = 1
+    for pos in range(a, z, max(1, (z - a) // 12)):
+        for bit in (0, 3, 7):
+            bad = pay.copy()
+            bad[pos] ^= 1 << bit
+            try:
+                want = O.block_masked_sum(g, bad, 8, w.n_pixels, np.array([q]), np.array([1]))
+            except O.MalformedStream:
+                want = None
+            res = oracle_resident(w, enc, payloads=[bad])
+            if want is None:
+                with pytest.raises(V.MalformedStream):
+                    image(res, m, 1)
+            else:
+                assert (image(res, m, 1)[0] == want.astype(np.uint64)).all()
+            res.free()
+
+
+def test_async_queries_and_finish(data):
+    w, x, enc = data("c2")
+    res = gpu_encode(w, x)
+    outs = []
+    for mname in ("bf", "adf"):
+        for k in (1, 2):
+            outs.append((mname, k, res.masked_sum(to_dev(w.masks[mname]), block_stride=k, wait=False)))
+    res.finish()
+    for mname, k, o in outs:
+        assert (V.as_unsigned(o).astype(np.uint64) == O.dense_masked_sum(x, w.masks[mname], None, k)).all()
+    res.free()
+
+
+def test_append_in_pieces(data):
+    w, x, enc = data("c2")
+    res = V.Resident.create((w.scan_rows, w.scan_cols), (w.det_rows, w.det_cols), w.dtype_bits)
+    xd = to_dev(x)
+    res.append(xd[: 3 * 512], 3)
+    res.append(xd[3 * 512: 4 * 512], 1)
+    res.append(xd[4 * 512:], 4)
+    for b, (g, p) in enumerate(export_all(res, w.n_blocks)):
+        assert (g == enc.groups[b]).all() and (p == enc.payloads[b]).all()
+    with pytest.raises(V.QemError):
+        res.append(xd[:512], 1)
+    res.free()
+
+
+def test_library_tables_equal_oracle():
+    f, a, c = V.model_tables()
+    f2, a2, c2 = O.models()
+    assert (f == f2).all() and (a == a2).all() and (c == c2).all()

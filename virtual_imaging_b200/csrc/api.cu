@@ -1,0 +1,791 @@
+// api.cu -- C ABI of libqem: the resident, its arenas, query planning on the
+// host side, per-stride baselines and the deferred error status.
+//
+// Page "Paired-count resident layout": "Operation pipeline" steps 1-6 and
+// "Contract" (virtual image dtype rule, malformed streams raise, queued
+// queries with a failed decode invalidating the incremental plan).
+#include <chrono>
+#include <cstring>
+#include <map>
+#include <thread>
+#include <vector>
+
+#include "qem_internal.h"
+
+using namespace qem;
+
+namespace {
+
+constexpr size_t kArenaMax = size_t(1) << 30;       // payload allocation unit
+constexpr size_t kBatchRawBytes = size_t(64) << 20; // raw counts encoded per batch (L2-sized)
+constexpr double kWaitSeconds = 60.0;
+
+enum BaseState { kNone = 0, kValid = 1, kTainted = 2 };
+
+struct Baseline {
+    uint8_t *d_mask = nullptr;
+    void *d_img = nullptr;
+    int out_bits = 0;
+    int state = kNone;
+    bool pending = false;     // written since the last successful finish
+};
+
+struct Arena {
+    uint8_t *p = nullptr;
+    size_t cap = 0;
+    size_t used = 0;
+};
+
+struct ProfEvent {
+    int kernel;
+    cudaEvent_t a, b;
+};
+
+}  // namespace
+
+struct qem_resident {
+    int device = 0;
+    int64_t scan_rows = 0, scan_cols = 0;
+    int det_rows = 0, det_cols = 0;
+    int bits = 8, w = 1;
+    int P = 0, G = 0;
+    int64_t B = 0, B_done = 0;
+    int n_valid = 0;
+    int out_bits_auto = 32;
+    int n_sm = 1;
+
+    uint8_t *d_valid = nullptr;
+    uint32_t *d_groups = nullptr;
+    unsigned long long *d_blk_ptr = nullptr;
+    uint32_t *d_blk_len = nullptr;
+    std::vector<uint64_t> blk_len;
+    std::vector<unsigned long long> blk_ptr;
+    std::vector<Arena> arenas;
+
+    uint32_t *d_dec = nullptr, *d_enc_sym = nullptr, *d_cost = nullptr, *d_amax = nullptr;
+    uint16_t *d_enc_slot = nullptr;
+
+    uint4 *d_desc = nullptr;
+    uint32_t *d_slots = nullptr;
+    size_t scratch_streams = 0;
+    unsigned long long *d_stats = nullptr;
+    uint32_t *h_len = nullptr;                  // pinned
+    unsigned long long *h_ptr = nullptr;        // pinned
+    size_t pinned_blocks = 0;
+
+    uint32_t *d_list = nullptr;
+    uint32_t *d_count = nullptr;
+    DevStatus *d_status = nullptr;
+    DevStatus *h_status = nullptr;              // pinned
+    std::map<int, Baseline> baselines;
+
+    uint64_t form_count[5] = {0, 0, 0, 0, 0};
+    uint64_t model_count[32] = {0};
+
+    bool prof = false;
+    std::vector<ProfEvent> events;
+    qem_profile_t prof_acc{};
+
+    Tables tables() const { return Tables{d_dec, d_enc_sym, d_enc_slot, d_cost, d_amax}; }
+    View view() const { return View{d_groups, d_blk_ptr, d_blk_len, d_valid, P, G, w, B}; }
+};
+
+namespace {
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return QEM_OK;
+    return e == cudaErrorMemoryAllocation ? QEM_ERR_OOM : QEM_ERR_CUDA;
+}
+
+#define QEM_CK(expr)                                   \
+    do {                                               \
+        const cudaError_t qem_e_ = (expr);             \
+        if (qem_e_ != cudaSuccess)                     \
+            return cuda_status(qem_e_);                \
+    } while (0)
+
+template <typename F>
+int timed(qem_resident *r, int kernel, cudaStream_t st, F &&launch)
+{
+    if (!r->prof)
+        return cuda_status(launch());
+    ProfEvent ev{kernel, nullptr, nullptr};
+    QEM_CK(cudaEventCreate(&ev.a));
+    QEM_CK(cudaEventCreate(&ev.b));
+    QEM_CK(cudaEventRecord(ev.a, st));
+    const cudaError_t e = launch();
+    QEM_CK(cudaEventRecord(ev.b, st));
+    r->events.push_back(ev);
+    return cuda_status(e);
+}
+
+// Wait for everything queued on `st` so far, with a time limit.
+int bounded_wait(cudaStream_t st)
+{
+    cudaEvent_t ev;
+    QEM_CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    cudaError_t e = cudaEventRecord(ev, st);
+    if (e != cudaSuccess) {
+        cudaEventDestroy(ev);
+        return cuda_status(e);
+    }
+    const auto t0 = std::chrono::steady_clock::now();
+    int rc = QEM_OK;
+    for (;;) {
+        e = cudaEventQuery(ev);
+        if (e == cudaSuccess)
+            break;
+        if (e != cudaErrorNotReady) {
+            rc = cuda_status(e);
+            break;
+        }
+        const double dt = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+        if (dt > kWaitSeconds) {
+            rc = QEM_ERR_TIMEOUT;
+            break;
+        }
+        std::this_thread::sleep_for(std::chrono::microseconds(dt < 0.01 ? 2 : 200));
+    }
+    cudaEventDestroy(ev);
+    return rc;
+}
+
+template <typename T>
+int dalloc(T **p, size_t bytes)
+{
+    void *q = nullptr;
+    QEM_CK(cudaMalloc(&q, bytes ? bytes : 16));
+    *p = static_cast<T *>(q);
+    return QEM_OK;
+}
+
+void release(qem_resident *r)
+{
+    for (auto &ev : r->events) {
+        cudaEventDestroy(ev.a);
+        cudaEventDestroy(ev.b);
+    }
+    for (auto &a : r->arenas)
+        cudaFree(a.p);
+    for (auto &kv : r->baselines) {
+        cudaFree(kv.second.d_mask);
+        cudaFree(kv.second.d_img);
+    }
+    cudaFree(r->d_valid);
+    cudaFree(r->d_groups);
+    cudaFree(r->d_blk_ptr);
+    cudaFree(r->d_blk_len);
+    cudaFree(r->d_dec);
+    cudaFree(r->d_enc_sym);
+    cudaFree(r->d_enc_slot);
+    cudaFree(r->d_cost);
+    cudaFree(r->d_amax);
+    cudaFree(r->d_desc);
+    cudaFree(r->d_slots);
+    cudaFree(r->d_stats);
+    cudaFree(r->d_list);
+    cudaFree(r->d_count);
+    cudaFree(r->d_status);
+    cudaFreeHost(r->h_len);
+    cudaFreeHost(r->h_ptr);
+    cudaFreeHost(r->h_status);
+    delete r;
+}
+
+int check_geometry(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t det_cols, int32_t bits)
+{
+    if (scan_rows <= 0 || scan_cols <= 0 || det_rows <= 0 || det_cols <= 0)
+        return QEM_ERR_ARG;
+    if ((scan_rows * scan_cols) % kScans != 0)
+        return QEM_ERR_ARG;
+    if (static_cast<int64_t>(det_rows) * det_cols >= (int64_t(1) << 24))
+        return QEM_ERR_ARG;
+    if (bits != 8 && bits != 16)
+        return QEM_ERR_ARG;
+    return QEM_OK;
+}
+
+int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t det_cols, int32_t bits,
+                  const uint8_t *valid, bool valid_on_host, cudaStream_t st, qem_resident **out)
+{
+    *out = nullptr;
+    int rc = check_geometry(scan_rows, scan_cols, det_rows, det_cols, bits);
+    if (rc)
+        return rc;
+    qem_resident *r = new qem_resident();
+    auto fail = [&](int code) {
+        release(r);
+        return code;
+    };
+    cudaGetDevice(&r->device);
+    cudaDeviceGetAttribute(&r->n_sm, cudaDevAttrMultiProcessorCount, r->device);
+    r->scan_rows = scan_rows;
+    r->scan_cols = scan_cols;
+    r->det_rows = det_rows;
+    r->det_cols = det_cols;
+    r->bits = bits;
+    r->w = bits / 8;
+    r->P = det_rows * det_cols;
+    r->G = (r->P + 31) / 32;
+    r->B = scan_rows * scan_cols / kScans;
+    r->blk_len.assign(static_cast<size_t>(r->B), 0);
+    r->blk_ptr.assign(static_cast<size_t>(r->B), 0);
+
+    std::vector<uint8_t> hv(static_cast<size_t>(r->P), 1);
+    if (valid) {
+        const cudaError_t e = valid_on_host
+                                  ? (std::memcpy(hv.data(), valid, hv.size()), cudaSuccess)
+                                  : cudaMemcpy(hv.data(), valid, hv.size(), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess)
+            return fail(cuda_status(e));
+    }
+    r->n_valid = 0;
+    for (auto &x : hv) {
+        x = x ? 1 : 0;
+        r->n_valid += x;
+    }
+    r->out_bits_auto = static_cast<uint64_t>(r->n_valid) * ((1ull << bits) - 1ull) > 0xFFFFFFFFull ? 64 : 32;
+
+    const HostTables &T = host_tables();
+    if ((rc = dalloc(&r->d_valid, hv.size())) || (rc = dalloc(&r->d_groups, size_t(r->B) * r->G * kGroupWords * 4)) ||
+        (rc = dalloc(&r->d_blk_ptr, size_t(r->B) * 8)) || (rc = dalloc(&r->d_blk_len, size_t(r->B) * 4)) ||
+        (rc = dalloc(&r->d_dec, sizeof(T.dec))) || (rc = dalloc(&r->d_enc_sym, sizeof(T.enc_sym))) ||
+        (rc = dalloc(&r->d_enc_slot, sizeof(T.enc_slot))) || (rc = dalloc(&r->d_cost, sizeof(T.cost))) ||
+        (rc = dalloc(&r->d_amax, kModels * 4)) || (rc = dalloc(&r->d_stats, (5 + kModels) * 8)) ||
+        (rc = dalloc(&r->d_list, size_t(r->P) * 4)) || (rc = dalloc(&r->d_count, 16)) ||
+        (rc = dalloc(&r->d_status, sizeof(DevStatus))))
+        return fail(rc);
+    if (cudaMallocHost(&r->h_status, sizeof(DevStatus)) != cudaSuccess)
+        return fail(QEM_ERR_OOM);
+    std::memset(r->h_status, 0, sizeof(DevStatus));
+    uint32_t amax[kModels];
+    for (int m = 0; m < kModels; ++m)
+        amax[m] = T.amax[m];
+    cudaError_t e = cudaSuccess;
+    auto up = [&](void *d, const void *h, size_t n) {
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, st);
+    };
+    up(r->d_valid, hv.data(), hv.size());
+    up(r->d_dec, T.dec, sizeof(T.dec));
+    up(r->d_enc_sym, T.enc_sym, sizeof(T.enc_sym));
+    up(r->d_enc_slot, T.enc_slot, sizeof(T.enc_slot));
+    up(r->d_cost, T.cost, sizeof(T.cost));
+    up(r->d_amax, amax, sizeof(amax));
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(r->d_stats, 0, (5 + kModels) * 8, st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(r->d_status, 0, sizeof(DevStatus), st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(r->d_groups, 0, size_t(r->B) * r->G * kGroupWords * 4, st);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(st);        // host staging above goes out of scope
+    if (e != cudaSuccess)
+        return fail(cuda_status(e));
+    *out = r;
+    return QEM_OK;
+}
+
+// Place a block of `len` bytes in an arena (new arena when the current is full).
+int place_block(qem_resident *r, int64_t b, uint64_t len, unsigned long long &ptr)
+{
+    const size_t need = static_cast<size_t>(len) + kArenaPad;
+    if (r->arenas.empty() || r->arenas.back().used + need > r->arenas.back().cap) {
+        const size_t bound_rest = static_cast<size_t>(r->B - b) * r->P * (2 + kScans * r->w) + kArenaPad;
+        size_t cap = bound_rest < kArenaMax ? bound_rest : kArenaMax;
+        if (cap < need)
+            cap = need;
+        cap = (cap + 255) & ~size_t(255);
+        Arena a;
+        void *p = nullptr;
+        QEM_CK(cudaMalloc(&p, cap));
+        a.p = static_cast<uint8_t *>(p);
+        a.cap = cap;
+        a.used = 0;
+        r->arenas.push_back(a);
+        QEM_CK(cudaMemset(a.p, 0, cap));
+    }
+    Arena &a = r->arenas.back();
+    ptr = reinterpret_cast<unsigned long long>(a.p + a.used);
+    a.used = (a.used + static_cast<size_t>(len) + 15) & ~size_t(15);
+    return QEM_OK;
+}
+
+int ensure_scratch(qem_resident *r, int nblk)
+{
+    const size_t streams = static_cast<size_t>(nblk) * r->P;
+    if (streams > r->scratch_streams) {
+        cudaFree(r->d_desc);
+        cudaFree(r->d_slots);
+        r->d_desc = nullptr;
+        r->d_slots = nullptr;
+        r->scratch_streams = 0;
+        int rc;
+        if ((rc = dalloc(&r->d_desc, streams * sizeof(uint4))) ||
+            (rc = dalloc(&r->d_slots, streams * kSlotWords * sizeof(uint32_t))))
+            return rc;
+        r->scratch_streams = streams;
+    }
+    if (static_cast<size_t>(nblk) > r->pinned_blocks) {
+        cudaFreeHost(r->h_len);
+        cudaFreeHost(r->h_ptr);
+        r->h_len = nullptr;
+        r->h_ptr = nullptr;
+        r->pinned_blocks = 0;
+        QEM_CK(cudaMallocHost(&r->h_len, static_cast<size_t>(nblk) * 4));
+        QEM_CK(cudaMallocHost(&r->h_ptr, static_cast<size_t>(nblk) * 8));
+        r->pinned_blocks = static_cast<size_t>(nblk);
+    }
+    return QEM_OK;
+}
+
+int collect_stats(qem_resident *r, cudaStream_t st)
+{
+    unsigned long long h[5 + kModels];
+    QEM_CK(cudaMemcpyAsync(h, r->d_stats, sizeof(h), cudaMemcpyDeviceToHost, st));
+    QEM_CK(cudaStreamSynchronize(st));
+    for (int i = 0; i < 5; ++i)
+        r->form_count[i] += h[i];
+    for (int m = 0; m < kModels; ++m)
+        r->model_count[m] += h[5 + m];
+    QEM_CK(cudaMemsetAsync(r->d_stats, 0, sizeof(h), st));
+    return QEM_OK;
+}
+
+int report_errors(qem_resident *r, cudaStream_t st)
+{
+    if (r->h_status->flags == 0u) {
+        for (auto &kv : r->baselines)
+            kv.second.pending = false;
+        return QEM_OK;
+    }
+    for (auto &kv : r->baselines)
+        if (kv.second.pending) {
+            kv.second.state = kTainted;
+            kv.second.pending = false;
+        }
+    const unsigned long long rows = r->h_status->rows, streams = r->h_status->streams;
+    std::memset(r->h_status, 0, sizeof(DevStatus));
+    r->h_status->rows = rows;
+    r->h_status->streams = streams;
+    QEM_CK(cudaMemcpyAsync(r->d_status, r->h_status, sizeof(DevStatus), cudaMemcpyHostToDevice, st));
+    QEM_CK(cudaStreamSynchronize(st));
+    return QEM_ERR_MALFORMED;
+}
+
+int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, void *d_out, int32_t *used,
+          int32_t wait, cudaStream_t st, bool delta)
+{
+    if (!r || !d_mask || !d_out || k < 1 || (reinterpret_cast<uintptr_t>(d_out) & 15u))
+        return QEM_ERR_ARG;
+    if (r->B_done != r->B)
+        return QEM_ERR_STATE;
+    int bits;
+    if (out_bits == 0)
+        bits = r->out_bits_auto;
+    else if (out_bits == 64)
+        bits = 64;
+    else if (out_bits == 32 && r->out_bits_auto == 32)
+        bits = 32;
+    else
+        return QEM_ERR_ARG;
+    const long long rows = (r->B + k - 1) / k;
+    const long long n_elems = rows * kScans;
+    const size_t out_bytes = static_cast<size_t>(n_elems) * (bits / 8);
+
+    Baseline &bl = r->baselines[k];
+    if (!bl.d_mask) {
+        int rc;
+        if ((rc = dalloc(&bl.d_mask, r->P)) || (rc = dalloc(&bl.d_img, static_cast<size_t>(n_elems) * 8)))
+            return rc;
+        QEM_CK(cudaMemsetAsync(bl.d_mask, 0, r->P, st));
+    }
+    int mode = 0;
+    if (delta) {
+        if (bl.state == kTainted)
+            return QEM_ERR_TAINTED;
+        if (bl.state == kValid && bl.out_bits == bits)
+            mode = 1;
+    }
+    int rc = timed(r, QEM_K_PLAN, st, [&] {
+        return launch_plan(d_mask, r->d_valid, bl.d_mask, r->P, mode, r->d_list, r->d_count, d_out, bl.d_img,
+                           n_elems, bits / 8, st);
+    });
+    if (rc)
+        return rc;
+    rc = timed(r, QEM_K_DECODE_REDUCE, st, [&] {
+        return launch_decode_reduce(r->view(), r->tables(), r->d_list, r->d_count, k, rows, d_out, bits / 8,
+                                    r->d_status, r->n_sm, st);
+    });
+    if (rc)
+        return rc;
+    rc = timed(r, QEM_K_FINALIZE, st, [&] { return launch_copy(bl.d_img, d_out, out_bytes, st); });
+    if (rc)
+        return rc;
+    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+    bl.state = kValid;
+    bl.out_bits = bits;
+    bl.pending = true;
+    if (used)
+        *used = bits;
+    if (wait) {
+        rc = bounded_wait(st);
+        if (rc)
+            return rc;
+        return report_errors(r, st);
+    }
+    return QEM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *qem_abi(void) { return "qem-pair-v1"; }
+
+const char *qem_status_string(int s)
+{
+    switch (s) {
+    case QEM_OK: return "ok";
+    case QEM_ERR_ARG: return "invalid argument";
+    case QEM_ERR_MALFORMED: return "malformed stream";
+    case QEM_ERR_CUDA: return "CUDA error";
+    case QEM_ERR_OOM: return "out of device memory";
+    case QEM_ERR_TIMEOUT: return "device wait timed out";
+    case QEM_ERR_TAINTED: return "delta baseline invalidated by a failed decode";
+    case QEM_ERR_STATE: return "resident not complete";
+    default: return "unknown status";
+    }
+}
+
+int qem_create(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t det_cols, int32_t dtype_bits,
+               const uint8_t *d_valid, void *stream, qem_resident **out)
+{
+    if (!out)
+        return QEM_ERR_ARG;
+    return make_resident(scan_rows, scan_cols, det_rows, det_cols, dtype_bits, d_valid, false,
+                         static_cast<cudaStream_t>(stream), out);
+}
+
+int qem_encode_append(qem_resident *r, const void *d_counts, int64_t n_blocks, void *stream)
+{
+    if (!r || !d_counts || n_blocks < 0 || r->B_done + n_blocks > r->B ||
+        (reinterpret_cast<uintptr_t>(d_counts) & static_cast<uintptr_t>(r->w - 1)))
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t block_raw = static_cast<size_t>(kScans) * r->P * r->w;
+    int64_t per = static_cast<int64_t>(kBatchRawBytes / block_raw);
+    if (per < 1)
+        per = 1;
+    if (per > n_blocks)
+        per = n_blocks > 0 ? n_blocks : 1;
+    int rc = ensure_scratch(r, static_cast<int>(per));
+    if (rc)
+        return rc;
+    const uint8_t *src = static_cast<const uint8_t *>(d_counts);
+    for (int64_t done = 0; done < n_blocks;) {
+        const int nb = static_cast<int>(n_blocks - done < per ? n_blocks - done : per);
+        const void *counts = src + static_cast<size_t>(done) * block_raw;
+        const int64_t b0 = r->B_done;
+        rc = timed(r, QEM_K_ENC_STREAMS, st, [&] {
+            return launch_enc_streams(counts, r->w, r->P, nb, r->tables(), r->d_desc, r->d_slots, r->d_stats, st);
+        });
+        if (rc)
+            return rc;
+        rc = timed(r, QEM_K_ENC_LAYOUT, st, [&] {
+            return launch_enc_layout(r->d_desc, r->P, r->G, nb, r->d_groups + size_t(b0) * r->G * kGroupWords,
+                                     r->d_blk_len + b0, st);
+        });
+        if (rc)
+            return rc;
+        QEM_CK(cudaMemcpyAsync(r->h_len, r->d_blk_len + b0, size_t(nb) * 4, cudaMemcpyDeviceToHost, st));
+        QEM_CK(cudaStreamSynchronize(st));
+        for (int i = 0; i < nb; ++i) {
+            unsigned long long ptr;
+            if ((rc = place_block(r, b0 + i, r->h_len[i], ptr)))
+                return rc;
+            r->h_ptr[i] = ptr;
+            r->blk_len[b0 + i] = r->h_len[i];
+            r->blk_ptr[b0 + i] = ptr;
+        }
+        QEM_CK(cudaMemcpyAsync(r->d_blk_ptr + b0, r->h_ptr, size_t(nb) * 8, cudaMemcpyHostToDevice, st));
+        rc = timed(r, QEM_K_ENC_COMPACT, st, [&] {
+            return launch_enc_compact(counts, r->w, r->P, nb, r->d_desc, r->d_slots, r->d_blk_ptr + b0, st);
+        });
+        if (rc)
+            return rc;
+        r->B_done += nb;
+        done += nb;
+    }
+    return collect_stats(r, st);
+}
+
+int qem_encode(const void *d_counts, int32_t dtype_bits, int64_t scan_rows, int64_t scan_cols, int32_t det_rows,
+               int32_t det_cols, const uint8_t *d_valid, void *stream, qem_resident **out)
+{
+    if (!out || !d_counts)
+        return QEM_ERR_ARG;
+    int rc = qem_create(scan_rows, scan_cols, det_rows, det_cols, dtype_bits, d_valid, stream, out);
+    if (rc)
+        return rc;
+    rc = qem_encode_append(*out, d_counts, (*out)->B, stream);
+    if (rc == QEM_OK)
+        rc = cuda_status(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    if (rc) {
+        release(*out);
+        *out = nullptr;
+    }
+    return rc;
+}
+
+int qem_masked_sum(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, void *d_out,
+                   int32_t *used, int32_t wait, void *stream)
+{
+    return query(r, d_mask, k, out_bits, d_out, used, wait, static_cast<cudaStream_t>(stream), false);
+}
+
+int qem_masked_sum_delta(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, void *d_out,
+                         int32_t *used, int32_t wait, void *stream)
+{
+    return query(r, d_mask, k, out_bits, d_out, used, wait, static_cast<cudaStream_t>(stream), true);
+}
+
+int qem_decode_blocks(qem_resident *r, int64_t first, int64_t n, void *d_out, int32_t wait, void *stream)
+{
+    if (!r || !d_out || first < 0 || n < 0 || first + n > r->B_done ||
+        (reinterpret_cast<uintptr_t>(d_out) & static_cast<uintptr_t>(r->w - 1)))
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n == 0)
+        return QEM_OK;
+    int rc = timed(r, QEM_K_DECODE_BLOCKS, st, [&] {
+        return launch_decode_blocks(r->view(), r->tables(), first, n, d_out, r->d_status, st);
+    });
+    if (rc)
+        return rc;
+    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+    if (wait) {
+        rc = bounded_wait(st);
+        if (rc)
+            return rc;
+        return report_errors(r, st);
+    }
+    return QEM_OK;
+}
+
+int qem_finish(qem_resident *r, void *stream)
+{
+    if (!r)
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+    const int rc = bounded_wait(st);
+    if (rc)
+        return rc;
+    return report_errors(r, st);
+}
+
+int qem_info(const qem_resident *r, qem_info_t *o)
+{
+    if (!r || !o)
+        return QEM_ERR_ARG;
+    std::memset(o, 0, sizeof(*o));
+    o->scan_rows = r->scan_rows;
+    o->scan_cols = r->scan_cols;
+    o->det_rows = r->det_rows;
+    o->det_cols = r->det_cols;
+    o->dtype_bits = r->bits;
+    o->n_pixels = r->P;
+    o->n_valid = r->n_valid;
+    o->out_bits_auto = r->out_bits_auto;
+    o->n_blocks = r->B;
+    o->n_blocks_encoded = r->B_done;
+    for (int64_t b = 0; b < r->B_done; ++b)
+        o->payload_bytes += r->blk_len[b];
+    o->group_bytes = static_cast<uint64_t>(r->B) * r->G * kGroupWords * 4;
+    uint64_t dev = o->group_bytes + r->B * 12 + r->P + r->P * 4;
+    for (auto &a : r->arenas)
+        dev += a.cap;
+    dev += r->scratch_streams * (sizeof(uint4) + kSlotWords * 4);
+    for (auto &kv : r->baselines)
+        dev += r->P + static_cast<uint64_t>((r->B + kv.first - 1) / kv.first) * kScans * 8;
+    dev += sizeof(HostTables);
+    o->device_bytes = dev;
+    for (int i = 0; i < 5; ++i)
+        o->form_count[i] = r->form_count[i];
+    for (int m = 0; m < kModels; ++m)
+        o->model_count[m] = r->model_count[m];
+    o->n_arenas = static_cast<int32_t>(r->arenas.size());
+    return QEM_OK;
+}
+
+int qem_query_counters(qem_resident *r, uint64_t *rows, uint64_t *streams, void *stream)
+{
+    if (!r)
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus h;
+    QEM_CK(cudaMemcpyAsync(&h, r->d_status, sizeof(h), cudaMemcpyDeviceToHost, st));
+    QEM_CK(cudaStreamSynchronize(st));
+    if (rows)
+        *rows = h.rows;
+    if (streams)
+        *streams = h.streams;
+    QEM_CK(cudaMemsetAsync(reinterpret_cast<uint8_t *>(r->d_status) + offsetof(DevStatus, rows), 0,
+                           2 * sizeof(unsigned long long), st));
+    QEM_CK(cudaStreamSynchronize(st));
+    return QEM_OK;
+}
+
+int qem_profile(qem_resident *r, int32_t enable)
+{
+    if (!r)
+        return QEM_ERR_ARG;
+    r->prof = enable != 0;
+    if (enable)
+        std::memset(&r->prof_acc, 0, sizeof(r->prof_acc));
+    return QEM_OK;
+}
+
+int qem_profile_read(qem_resident *r, qem_profile_t *out)
+{
+    if (!r || !out)
+        return QEM_ERR_ARG;
+    for (auto &ev : r->events) {
+        QEM_CK(cudaEventSynchronize(ev.b));
+        float ms = 0.f;
+        QEM_CK(cudaEventElapsedTime(&ms, ev.a, ev.b));
+        r->prof_acc.ms[ev.kernel] += ms;
+        r->prof_acc.launches[ev.kernel] += 1;
+        cudaEventDestroy(ev.a);
+        cudaEventDestroy(ev.b);
+    }
+    r->events.clear();
+    *out = r->prof_acc;
+    return QEM_OK;
+}
+
+void qem_free(qem_resident *r)
+{
+    if (!r)
+        return;
+    cudaDeviceSynchronize();
+    release(r);
+}
+
+int qem_block_bytes(const qem_resident *r, int64_t b, uint64_t *nbytes)
+{
+    if (!r || !nbytes || b < 0 || b >= r->B_done)
+        return QEM_ERR_ARG;
+    *nbytes = r->blk_len[b];
+    return QEM_OK;
+}
+
+int qem_export_block(const qem_resident *r, int64_t b, uint32_t *h_groups, uint8_t *h_payload, void *stream)
+{
+    if (!r || b < 0 || b >= r->B_done)
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (h_groups)
+        QEM_CK(cudaMemcpyAsync(h_groups, r->d_groups + size_t(b) * r->G * kGroupWords,
+                               size_t(r->G) * kGroupWords * 4, cudaMemcpyDeviceToHost, st));
+    if (h_payload && r->blk_len[b])
+        QEM_CK(cudaMemcpyAsync(h_payload, reinterpret_cast<const void *>(r->blk_ptr[b]), r->blk_len[b],
+                               cudaMemcpyDeviceToHost, st));
+    QEM_CK(cudaStreamSynchronize(st));
+    return QEM_OK;
+}
+
+int qem_import(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t det_cols, int32_t dtype_bits,
+               const uint32_t *h_groups, const uint8_t *h_payload, const uint64_t *h_block_off,
+               const uint8_t *h_valid, void *stream, qem_resident **out)
+{
+    if (!out || !h_groups || !h_payload || !h_block_off)
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    qem_resident *r = nullptr;
+    int rc = make_resident(scan_rows, scan_cols, det_rows, det_cols, dtype_bits, h_valid, true, st, &r);
+    if (rc)
+        return rc;
+    auto fail = [&](int code) {
+        release(r);
+        *out = nullptr;
+        return code;
+    };
+    const uint64_t total = h_block_off[r->B] - h_block_off[0];
+    Arena a;
+    a.cap = (static_cast<size_t>(total) + kArenaPad + 255) & ~size_t(255);
+    void *p = nullptr;
+    if (cudaMalloc(&p, a.cap) != cudaSuccess)
+        return fail(QEM_ERR_OOM);
+    a.p = static_cast<uint8_t *>(p);
+    a.used = total;
+    r->arenas.push_back(a);
+    cudaError_t e = cudaMemset(a.p, 0, a.cap);
+    if (e == cudaSuccess && total)
+        e = cudaMemcpy(a.p, h_payload + h_block_off[0], total, cudaMemcpyHostToDevice);
+    std::vector<uint32_t> lens(static_cast<size_t>(r->B));
+    for (int64_t b = 0; b < r->B; ++b) {
+        r->blk_ptr[b] = reinterpret_cast<unsigned long long>(a.p + (h_block_off[b] - h_block_off[0]));
+        r->blk_len[b] = h_block_off[b + 1] - h_block_off[b];
+        lens[b] = static_cast<uint32_t>(r->blk_len[b]);
+        // statistics from the headers, as the encoder would have counted them
+        const uint32_t *g = h_groups + size_t(b) * r->G * kGroupWords;
+        const uint8_t *pl = h_payload + h_block_off[b];
+        for (int px = 0; px < r->P; ++px) {
+            const uint32_t *rec = g + size_t(px >> 5) * kGroupWords;
+            const int j = px & 31;
+            const uint32_t e1 = (rec[1 + j / 2] >> (16 * (j & 1))) & 0xFFFFu;
+            const uint32_t e0 = j ? (rec[1 + (j - 1) / 2] >> (16 * ((j - 1) & 1))) & 0xFFFFu : 0u;
+            const uint64_t st0 = uint64_t(rec[0]) + e0;
+            if (e1 <= e0 || st0 + 2 > r->blk_len[b]) {
+                r->form_count[0] += e1 == e0;
+                continue;
+            }
+            const int form = pl[st0] & 7;
+            if (form >= 1 && form <= 4) {
+                r->form_count[form] += 1;
+                if (form == kPaired)
+                    r->model_count[(pl[st0] >> 3) & 31] += 1;
+            }
+        }
+    }
+    if (e == cudaSuccess)
+        e = cudaMemcpy(r->d_groups, h_groups, size_t(r->B) * r->G * kGroupWords * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(r->d_blk_ptr, r->blk_ptr.data(), size_t(r->B) * 8, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(r->d_blk_len, lens.data(), size_t(r->B) * 4, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess)
+        return fail(cuda_status(e));
+    r->B_done = r->B;
+    *out = r;
+    return QEM_OK;
+}
+
+int qem_model_tables(uint16_t *h_freq, uint8_t *h_amax, uint32_t *h_cost)
+{
+    const HostTables &T = host_tables();
+    if (h_freq)
+        std::memcpy(h_freq, T.freq, sizeof(T.freq));
+    if (h_amax)
+        std::memcpy(h_amax, T.amax, sizeof(T.amax));
+    if (h_cost)
+        std::memcpy(h_cost, T.cost, sizeof(T.cost));
+    return QEM_OK;
+}
+
+int qem_generate_counts(void *d_out, int32_t dtype_bits, uint64_t seed, int64_t scan0, int64_t n_scans,
+                        int32_t n_pixels, const uint32_t *d_pixel_class, const uint32_t *d_class_desc,
+                        const uint64_t *d_thresholds, void *stream)
+{
+    if (!d_out || !d_pixel_class || !d_class_desc || !d_thresholds || n_scans < 0 || n_pixels <= 0 ||
+        (dtype_bits != 8 && dtype_bits != 16))
+        return QEM_ERR_ARG;
+    return cuda_status(launch_generate(d_out, dtype_bits, seed, scan0, n_scans, n_pixels, d_pixel_class,
+                                       d_class_desc, d_thresholds, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,1165 @@
+// kernels.cu -- sm_100a kernels of the paired-count resident.
+//
+// Page "Paired-count resident layout":
+//  * "Operation pipeline" step 2 -- per-pixel 512-scan streams coded as count
+//    pairs with 1024-state tANS from 32 Poisson pair models; empty, constant,
+//    sparse and incompressible forms; grouped offsets (k_enc_streams,
+//    k_enc_layout, k_enc_compact);
+//  * step 4 -- a mask (or its difference from the previous mask) is turned
+//    into a pixel list (k_plan) and the streams are decoded one thread per
+//    stream with a 64-bit bit reservoir refilled four bytes at a time once per
+//    three coded pairs, reduced warp-wide per 32 scans into exact integer
+//    virtual images, optionally over every k-th block only (k_decode_reduce);
+//  * step 6 -- whole blocks decode back to native patterns (k_decode_blocks).
+// Bit-level choices follow the library's spec qem-pair-v1 (S1-S7).
+//
+// No kernel traps or asserts: malformed input sets flags in DevStatus and the
+// affected lane contributes zeros.  Every loop has a fixed trip count.
+#include <cstdio>
+#include <type_traits>
+
+#include "qem_internal.h"
+
+namespace qem {
+namespace {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void report(DevStatus *st, uint32_t flag, long long b, int p)
+{
+    atomicOr(&st->flags, flag);
+    if (atomicCAS(&st->have_first, 0u, 1u) == 0u) {
+        st->first_block = static_cast<uint32_t>(b);
+        st->first_pixel = static_cast<uint32_t>(p);
+    }
+}
+
+// Forward LSB-first bit reader over aligned 32-bit little-endian words: a
+// 64-bit reservoir `res` holding `n` valid bits.  Loads never pass `last`
+// (the aligned word holding the stream's final byte, plus one), so a
+// malformed stream reads repeated bytes inside its arena instead of running
+// off the end; the caller's length checks then reject it.
+struct Bits {
+    const uint32_t *wp;
+    const uint32_t *last;
+    const uint32_t *first;
+    uint64_t res;
+    int n;
+    int lead;      // bits of the first word before the stream start
+
+    __device__ __forceinline__ void init(const uint8_t *p, const uint8_t *end)
+    {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+        first = reinterpret_cast<const uint32_t *>(a & ~static_cast<uintptr_t>(3));
+        last = reinterpret_cast<const uint32_t *>((reinterpret_cast<uintptr_t>(end) + 3) &
+                                                  ~static_cast<uintptr_t>(3));
+        lead = static_cast<int>(a & 3) * 8;
+        res = __ldg(first) >> lead;
+        n = 32 - lead;
+        wp = first + 1;
+    }
+    __device__ __forceinline__ void refill()
+    {
+        const uint32_t *q = wp < last ? wp : last;
+        res |= static_cast<uint64_t>(__ldg(q)) << n;
+        n += 32;
+        ++wp;
+    }
+    __device__ __forceinline__ uint32_t get(int nb)
+    {
+        const uint32_t v = static_cast<uint32_t>(res) & ((1u << nb) - 1u);
+        res >>= nb;
+        n -= nb;
+        return v;
+    }
+    // bits consumed since init
+    __device__ __forceinline__ long long consumed() const
+    {
+        return 32ll * (wp - first) - lead - n;
+    }
+};
+
+__device__ __forceinline__ uint32_t load_native(const uint8_t *p, int w)
+{
+    return w == 2 ? static_cast<uint32_t>(__ldg(p)) | (static_cast<uint32_t>(__ldg(p + 1)) << 8)
+                  : static_cast<uint32_t>(__ldg(p));
+}
+
+// Parsed stream (spec S2/S3) with its readers.
+struct Stream {
+    int form;            // Form, kEmpty also for inactive or rejected lanes
+    int model;
+    int shift;
+    uint32_t base;
+    uint32_t c;          // constant value / sparse count
+    uint32_t x;          // tANS state minus 1024
+    const uint8_t *s;
+    uint32_t len;
+    uint32_t tans_len;   // paired: bytes of the tANS section
+    Bits bt;             // paired: tANS section; literal: values; sparse: positions
+    Bits br;             // paired: raw section; sparse: values
+};
+
+// Locate stream (b, p) through its group record and check the offsets (S1, S7).
+__device__ __forceinline__ bool locate(const View &v, long long b, int p, const uint8_t *&s,
+                                       uint32_t &len, DevStatus *st)
+{
+    const uint32_t *rec = v.groups + (static_cast<long long>(b) * v.G + (p >> 5)) * kGroupWords;
+    const int j = p & 31;
+    const uint32_t base = __ldg(rec);
+    const uint32_t w1 = __ldg(rec + 1 + (j >> 1));
+    const uint32_t e1 = (j & 1) ? (w1 >> 16) : (w1 & 0xFFFFu);
+    uint32_t e0 = 0;
+    if (j) {
+        const uint32_t w0 = __ldg(rec + 1 + ((j - 1) >> 1));
+        e0 = ((j - 1) & 1) ? (w0 >> 16) : (w0 & 0xFFFFu);
+    }
+    const uint32_t blen = __ldg(v.blk_len + b);
+    if (e1 < e0 || static_cast<uint64_t>(base) + e1 > blen) {
+        report(st, kErrOffsets, b, p);
+        return false;
+    }
+    s = reinterpret_cast<const uint8_t *>(__ldg(v.blk_ptr + b)) + base + e0;
+    len = e1 - e0;
+    return true;
+}
+
+// Parse the header and set the readers up; false (after reporting) if malformed.
+__device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
+{
+    if (S.len == 0) {
+        S.form = kEmpty;
+        return true;
+    }
+    if (S.len < 2) {
+        report(st, kErrLength, b, p);
+        return false;
+    }
+    const uint32_t hdr = static_cast<uint32_t>(__ldg(S.s)) | (static_cast<uint32_t>(__ldg(S.s + 1)) << 8);
+    if (hdr >> 13) {
+        report(st, kErrReserved, b, p);
+        return false;
+    }
+    S.form = static_cast<int>(hdr & 7);
+    S.model = static_cast<int>((hdr >> 3) & 31);
+    S.shift = static_cast<int>((hdr >> 8) & 15);
+    const int has_base = static_cast<int>((hdr >> 12) & 1);
+    if (S.form < kConstant || S.form > kLiteral) {
+        report(st, kErrForm, b, p);
+        return false;
+    }
+    if (S.form != kPaired && (S.model | S.shift | has_base)) {
+        report(st, kErrFields, b, p);
+        return false;
+    }
+    const uint8_t *end = S.s + S.len;
+    if (S.form == kConstant) {
+        if (S.len != static_cast<uint32_t>(2 + w)) {
+            report(st, kErrLength, b, p);
+            return false;
+        }
+        S.c = load_native(S.s + 2, w);
+        if (S.c == 0) {
+            report(st, kErrConstant, b, p);
+            return false;
+        }
+        return true;
+    }
+    if (S.form == kLiteral) {
+        if (S.len != static_cast<uint32_t>(2 + 512 * w)) {
+            report(st, kErrLength, b, p);
+            return false;
+        }
+        S.bt.init(S.s + 2, end);
+        return true;
+    }
+    if (S.form == kSparse) {
+        if (S.len < 3) {
+            report(st, kErrLength, b, p);
+            return false;
+        }
+        S.c = static_cast<uint32_t>(__ldg(S.s + 2)) + 1u;
+        const uint32_t pbytes = (9u * S.c + 7u) / 8u;
+        if (S.len != 3u + pbytes + S.c * static_cast<uint32_t>(w)) {
+            report(st, kErrLength, b, p);
+            return false;
+        }
+        S.bt.init(S.s + 3, end);
+        S.br.init(S.s + 3 + pbytes, end);
+        return true;
+    }
+    // paired
+    if (S.shift > 8 * w - 4) {
+        report(st, kErrFields, b, p);
+        return false;
+    }
+    uint32_t off = 2;
+    S.base = 0;
+    if (has_base) {
+        if (S.len < off + static_cast<uint32_t>(w)) {
+            report(st, kErrLength, b, p);
+            return false;
+        }
+        S.base = load_native(S.s + off, w);
+        off += static_cast<uint32_t>(w);
+    }
+    const uint32_t raw_off = off;
+    off += 64u * static_cast<uint32_t>(S.shift);
+    if (S.len < off + 2u) {
+        report(st, kErrLength, b, p);
+        return false;
+    }
+    S.tans_len = S.len - off;
+    S.br.init(S.s + raw_off, end);
+    S.bt.init(S.s + off, end);
+    if (S.bt.n < 10)
+        S.bt.refill();
+    S.x = S.bt.get(10);
+    return true;
+}
+
+// End-of-stream checks of a paired stream (S5/S7): final state 1024, section
+// length exactly ceil(T/8), zero pad bits.
+__device__ bool close_paired(Stream &S, long long b, int p, DevStatus *st)
+{
+    if (S.x != 0) {
+        report(st, kErrState, b, p);
+        return false;
+    }
+    const long long T = S.bt.consumed();
+    if ((T + 7) / 8 != static_cast<long long>(S.tans_len)) {
+        report(st, kErrLength, b, p);
+        return false;
+    }
+    const int pad = static_cast<int>(8ll * S.tans_len - T);
+    if (pad) {
+        if (S.bt.n < pad)
+            S.bt.refill();
+        if (S.bt.get(pad) != 0u) {
+            report(st, kErrPad, b, p);
+            return false;
+        }
+    }
+    return true;
+}
+
+// One tANS decode step with no raw bits: returns the table entry.
+__device__ __forceinline__ uint32_t tans_step(Stream &S, const uint32_t *dec)
+{
+    const uint32_t ent = dec[S.x];
+    const int nb = static_cast<int>((ent >> 10) & 15u);
+    S.x = (ent & 1023u) + S.bt.get(nb);
+    return ent;
+}
+
+// Decode 16 pairs (32 scans) of a paired stream into values v[32] (general
+// path: base and raw low bits).  Refill policy: the tANS reservoir is topped up
+// before pairs 0, 3, 6, 9, 12, 15 of the segment (<= 30 bits per 3 pairs);
+// the raw reservoir whenever it holds fewer than 2*shift bits.
+__device__ __forceinline__ void paired_segment(Stream &S, const uint32_t *dec, uint32_t (&v)[32],
+                                               uint32_t &over)
+{
+    const uint32_t mask = (1u << S.shift) - 1u;
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+        if (jj % 3 == 0 && S.bt.n < 30)
+            S.bt.refill();
+        if (S.br.n < 2 * S.shift)
+            S.br.refill();
+        const uint32_t ent = tans_step(S, dec);
+        const uint32_t lo = S.br.get(2 * S.shift);
+        const uint32_t va = S.base + ((((ent >> 16) & 0xFFu) << S.shift) | (lo & mask));
+        const uint32_t vb = S.base + (((ent >> 24) << S.shift) | ((lo >> S.shift) & mask));
+        over |= va | vb;
+        v[2 * jj] = va;
+        v[2 * jj + 1] = vb;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// synthetic generator (a1, bench/test input only)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_generate(T *__restrict__ out, uint64_t seed, int64_t scan0, int64_t n_scans, int P,
+                           const uint32_t *__restrict__ pclass, const uint4 *__restrict__ desc,
+                           const uint64_t *__restrict__ thr, uint32_t dmax)
+{
+    for (int64_t s = blockIdx.y; s < n_scans; s += gridDim.y) {
+        for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
+            const uint64_t idx = static_cast<uint64_t>(scan0 + s) * static_cast<uint64_t>(P) +
+                                 static_cast<uint64_t>(p) + 1ull;
+            uint64_t z = seed + idx * 0x9E3779B97F4A7C15ull;
+            z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+            z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+            z = z ^ (z >> 31);
+            const uint4 d = desc[pclass[p]];
+            uint32_t val;
+            if (d.x == 0u) {
+                const uint64_t u = z >> 11;
+                const uint64_t *t = thr + d.y;
+                int lo = 0, hi = static_cast<int>(d.z) - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (u >= __ldg(t + mid))
+                        lo = mid + 1;
+                    else
+                        hi = mid;
+                }
+                val = static_cast<uint32_t>(lo < 0 ? 0 : lo);
+            } else if (d.x == 1u) {
+                val = static_cast<uint32_t>(z) & dmax;
+            } else {
+                val = d.w;
+            }
+            out[s * P + p] = static_cast<T>(val < dmax ? val : dmax);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// encoder (a2-a4)
+// ---------------------------------------------------------------------------
+constexpr int kEncThreads = 256;
+
+// a2+a3: per stream (one thread): statistics, base/shift, hi histogram, model
+// selection (spec S6), backward tANS pass writing the section into this
+// stream's scratch slot from the top down (so the decoder reads it forward),
+// and the form decision.  desc: x = length, y = header | T << 16,
+// z = base (or constant value) | nnz << 16, w = offset (filled by layout).
+template <typename T>
+__global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict__ counts, int P, int nblk,
+                                                            Tables tb, uint4 *__restrict__ desc,
+                                                            uint32_t *__restrict__ slots,
+                                                            unsigned long long *__restrict__ stats)
+{
+    constexpr uint32_t W = sizeof(T);
+    __shared__ uint32_t s_cost[kModels * 16];
+    __shared__ uint32_t s_amax[kModels];
+    __shared__ uint16_t s_hist[16][kEncThreads];
+    __shared__ unsigned int s_stats[5 + kModels];
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kModels * 16; i += kEncThreads)
+        s_cost[i] = tb.cost[i];
+    if (tid < kModels)
+        s_amax[tid] = tb.amax[tid];
+    if (tid < 5 + kModels)
+        s_stats[tid] = 0;
+    __syncthreads();
+
+    const long long sid = static_cast<long long>(blockIdx.x) * kEncThreads + tid;
+    if (sid < static_cast<long long>(nblk) * P) {
+        const int b = static_cast<int>(sid / P);
+        const int p = static_cast<int>(sid - static_cast<long long>(b) * P);
+        const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
+
+        uint32_t nnz = 0, mn = 0xFFFFFFFFu, mx = 0;
+        {
+            const T *q = col;
+#pragma unroll 8
+            for (int i = 0; i < kScans; ++i, q += P) {
+                const uint32_t v = *q;
+                nnz += v != 0u;
+                mn = min(mn, v);
+                mx = max(mx, v);
+            }
+        }
+        uint4 d = make_uint4(0u, 0u, 0u, 0u);
+        int form = kEmpty, model = -1;
+        if (nnz == 0u) {
+            form = kEmpty;
+        } else if (mn == mx) {
+            form = kConstant;
+            d.x = 2u + W;
+            d.y = kConstant;
+            d.z = mn;
+        } else {
+            const uint32_t lit = 2u + 512u * W;
+            const uint32_t sparse = nnz <= 256u ? 3u + (9u * nnz + 7u) / 8u + nnz * W : 0xFFFFFFFFu;
+            const uint32_t has_base = mn > 0u ? 1u : 0u;
+            const uint32_t base = has_base ? mn : 0u;
+            const int span_bits = 32 - __clz(static_cast<int>(mx - base));
+            const int shift = span_bits > 4 ? span_bits - 4 : 0;
+
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+                s_hist[v][tid] = 0;
+            {
+                const T *q = col;
+#pragma unroll 8
+                for (int i = 0; i < kScans; ++i, q += P)
+                    s_hist[(static_cast<uint32_t>(*q) - base) >> shift][tid] += 1;
+            }
+            const uint32_t maxhi = (mx - base) >> shift;
+            uint32_t h[16];
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+                h[v] = s_hist[v][tid];
+            uint32_t best = 0xFFFFFFFFu;
+            model = kModels - 1;
+            for (int m = 0; m < kModels; ++m) {
+                if (s_amax[m] < maxhi)
+                    continue;
+                uint32_t c = 0;
+#pragma unroll
+                for (int v = 0; v < 16; ++v)
+                    c += h[v] * s_cost[m * 16 + v];
+                if (c < best) {
+                    best = c;
+                    model = m;
+                }
+            }
+
+            // backward tANS pass, chunks prepended at the low end of `acc`
+            const uint32_t *esym = tb.enc_sym + model * 256;
+            const uint16_t *eslot = tb.enc_slot + model * kStates;
+            uint32_t *slot = slots + static_cast<size_t>(sid) * kSlotWords;
+            int wi = kSlotWords - 1;
+            uint64_t acc = 0;
+            int nacc = 0;
+            uint32_t Tbits = 10;
+            uint32_t X = kStates;
+            const T *q = col + static_cast<size_t>(kScans - 2) * P;
+            for (int j = kPairs - 1; j >= 0; --j, q -= 2 * static_cast<size_t>(P)) {
+                const uint32_t a = (static_cast<uint32_t>(q[0]) - base) >> shift;
+                const uint32_t bb = (static_cast<uint32_t>(q[P]) - base) >> shift;
+                const uint32_t es = __ldg(esym + a + 16u * bb);
+                const uint32_t f = es & 0x7FFu;
+                const uint32_t cum = (es >> 11) & 0x7FFu;
+                const uint32_t k0 = es >> 22;
+                const uint32_t k = k0 - ((X >> k0) < f ? 1u : 0u);
+                const uint32_t chunk = X & ((1u << k) - 1u);
+                const uint32_t y = X >> k;
+                X = kStates + __ldg(eslot + cum + (y - f));
+                acc = (acc << k) | chunk;
+                nacc += static_cast<int>(k);
+                Tbits += k;
+                if (nacc >= 32) {
+                    slot[wi--] = static_cast<uint32_t>(acc >> (nacc - 32));
+                    nacc -= 32;
+                }
+            }
+            acc = (acc << 10) | (X - kStates);
+            nacc += 10;
+            if (nacc >= 32) {
+                slot[wi--] = static_cast<uint32_t>(acc >> (nacc - 32));
+                nacc -= 32;
+            }
+            if (nacc > 0)
+                slot[wi] = static_cast<uint32_t>(acc << (32 - nacc));
+
+            const uint32_t paired = 2u + has_base * W + 64u * static_cast<uint32_t>(shift) + (Tbits + 7u) / 8u;
+            uint32_t size;
+            if (sparse <= paired + 1u) {
+                form = kSparse;
+                size = sparse;
+            } else {
+                form = kPaired;
+                size = paired;
+            }
+            if (size >= lit) {
+                form = kLiteral;
+                size = lit;
+            }
+            d.x = size;
+            if (form == kPaired)
+                d.y = static_cast<uint32_t>(kPaired) | (static_cast<uint32_t>(model) << 3) |
+                      (static_cast<uint32_t>(shift) << 8) | (has_base << 12) | (Tbits << 16);
+            else
+                d.y = static_cast<uint32_t>(form);
+            d.z = base | (nnz << 16);
+        }
+        desc[sid] = d;
+        atomicAdd(&s_stats[form], 1u);
+        if (form == kPaired)
+            atomicAdd(&s_stats[5 + model], 1u);
+    }
+    __syncthreads();
+    if (tid < 5 + kModels && s_stats[tid])
+        atomicAdd(stats + tid, static_cast<unsigned long long>(s_stats[tid]));
+}
+
+constexpr int kLayoutThreads = 1024;
+
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t x, uint32_t *s_warp, uint32_t &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o)
+            inc += y;
+    }
+    if (lane == 31)
+        s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        uint32_t v = lane < nw ? s_warp[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, v, o);
+            if (lane >= o)
+                v += y;
+        }
+        if (lane < nw)
+            s_warp[lane] = v;          // inclusive warp prefix
+    }
+    __syncthreads();
+    total = s_warp[(blockDim.x >> 5) - 1];
+    const uint32_t before = warp ? s_warp[warp - 1] : 0u;
+    return before + inc - x;
+}
+
+// a4 (first half): per block, exclusive scan of stream lengths in pixel order
+// -> per-stream offsets (desc.w), block length, and the group records (S1).
+__global__ void __launch_bounds__(kLayoutThreads) k_enc_layout(uint4 *__restrict__ desc, int P, int G,
+                                                              uint32_t *__restrict__ groups,
+                                                              uint32_t *__restrict__ blk_len)
+{
+    __shared__ uint32_t s_warp[32];
+    const int b = blockIdx.x;
+    uint4 *d = desc + static_cast<size_t>(b) * P;
+    const int per = (P + kLayoutThreads - 1) / kLayoutThreads;
+    const int p0 = min(P, static_cast<int>(threadIdx.x) * per);
+    const int p1 = min(P, p0 + per);
+    uint32_t local = 0;
+    for (int p = p0; p < p1; ++p)
+        local += d[p].x;
+    uint32_t total;
+    uint32_t run = block_exclusive_scan(local, s_warp, total);
+    for (int p = p0; p < p1; ++p) {
+        d[p].w = run;
+        run += d[p].x;
+    }
+    if (threadIdx.x == 0)
+        blk_len[b] = total;
+    __syncthreads();
+    uint32_t *gb = groups + static_cast<size_t>(b) * G * kGroupWords;
+    for (int g = threadIdx.x; g < G; g += kLayoutThreads) {
+        uint32_t *rec = gb + static_cast<size_t>(g) * kGroupWords;
+        const uint32_t base = d[32 * g].w;
+        rec[0] = base;
+        uint32_t end = 0;
+        for (int j = 0; j < 32; j += 2) {
+            uint32_t lo, hi;
+            const int pa = 32 * g + j;
+            if (pa < P)
+                end = d[pa].w + d[pa].x - base;
+            lo = end;
+            if (pa + 1 < P)
+                end = d[pa + 1].w + d[pa + 1].x - base;
+            hi = end;
+            rec[1 + j / 2] = lo | (hi << 16);
+        }
+    }
+}
+
+// a4 (second half): write every stream's bytes at blk_dst[b] + offset.
+template <typename T>
+__global__ void __launch_bounds__(256) k_enc_compact(const T *__restrict__ counts, int P, int nblk,
+                                                    const uint4 *__restrict__ desc,
+                                                    const uint32_t *__restrict__ slots,
+                                                    const unsigned long long *__restrict__ blk_dst)
+{
+    constexpr uint32_t W = sizeof(T);
+    const long long sid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (sid >= static_cast<long long>(nblk) * P)
+        return;
+    const uint4 d = desc[sid];
+    if (d.x == 0u)
+        return;
+    const int b = static_cast<int>(sid / P);
+    const int p = static_cast<int>(sid - static_cast<long long>(b) * P);
+    const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
+    uint8_t *o = reinterpret_cast<uint8_t *>(blk_dst[b]) + d.w;
+    const uint32_t hdr = d.y & 0xFFFFu;
+    const int form = static_cast<int>(hdr & 7u);
+    o[0] = static_cast<uint8_t>(hdr & 0xFFu);
+    o[1] = static_cast<uint8_t>(hdr >> 8);
+    uint32_t k = 2;
+    auto put = [&](uint32_t v) {
+        o[k++] = static_cast<uint8_t>(v & 0xFFu);
+        if (W == 2)
+            o[k++] = static_cast<uint8_t>(v >> 8);
+    };
+    if (form == kConstant) {
+        put(d.z & 0xFFFFu);
+    } else if (form == kLiteral) {
+        const T *q = col;
+        for (int i = 0; i < kScans; ++i, q += P)
+            put(*q);
+    } else if (form == kSparse) {
+        const uint32_t nnz = d.z >> 16;
+        o[k++] = static_cast<uint8_t>(nnz - 1u);
+        uint32_t acc = 0;
+        int nacc = 0;
+        const T *q = col;
+        for (int i = 0; i < kScans; ++i, q += P) {
+            if (*q) {
+                acc |= static_cast<uint32_t>(i) << nacc;
+                nacc += 9;
+                while (nacc >= 8) {
+                    o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                    acc >>= 8;
+                    nacc -= 8;
+                }
+            }
+        }
+        if (nacc > 0)
+            o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+        q = col;
+        for (int i = 0; i < kScans; ++i, q += P)
+            if (*q)
+                put(*q);
+    } else {
+        const int shift = static_cast<int>((hdr >> 8) & 15u);
+        const uint32_t base = d.z & 0xFFFFu;
+        if ((hdr >> 12) & 1u)
+            put(base);
+        if (shift) {
+            const uint32_t mask = (1u << shift) - 1u;
+            uint32_t acc = 0;
+            int nacc = 0;
+            const T *q = col;
+            for (int i = 0; i < kScans; ++i, q += P) {
+                acc |= ((static_cast<uint32_t>(*q) - base) & mask) << nacc;
+                nacc += shift;
+                while (nacc >= 8) {
+                    o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                    acc >>= 8;
+                    nacc -= 8;
+                }
+            }
+        }
+        const uint32_t Tbits = d.y >> 16;
+        const uint32_t *sl = slots + static_cast<size_t>(sid) * kSlotWords;
+        const int nbytes = static_cast<int>((Tbits + 7u) / 8u);
+        const int o0 = 32 * kSlotWords - static_cast<int>(Tbits);
+        for (int q = 0; q < nbytes; ++q) {
+            const int bp = o0 + 8 * q;
+            const int wi = bp >> 5;
+            const uint64_t x = static_cast<uint64_t>(sl[wi]) |
+                               (wi + 1 < kSlotWords ? static_cast<uint64_t>(sl[wi + 1]) << 32 : 0ull);
+            o[k++] = static_cast<uint8_t>((x >> (bp & 31)) & 0xFFu);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a5: plan
+// ---------------------------------------------------------------------------
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict__ mask,
+                                                      const uint8_t *__restrict__ valid,
+                                                      uint8_t *__restrict__ base_mask, int P, int mode,
+                                                      uint32_t *__restrict__ list, uint32_t *__restrict__ count,
+                                                      uint4 *__restrict__ out, const uint4 *__restrict__ base_img,
+                                                      long long n_vec)
+{
+    if (blockIdx.x == 0) {
+        __shared__ uint32_t s_warp[32];
+        const int per = (P + kPlanThreads - 1) / kPlanThreads;
+        const int p0 = min(P, static_cast<int>(threadIdx.x) * per);
+        const int p1 = min(P, p0 + per);
+        uint32_t local = 0;
+        for (int p = p0; p < p1; ++p) {
+            const bool ok = valid[p] != 0;
+            const bool nw = ok && mask[p] != 0;
+            const bool od = ok && base_mask[p] != 0;
+            local += mode == 0 ? nw : (nw != od);
+        }
+        uint32_t total;
+        uint32_t pos = block_exclusive_scan(local, s_warp, total);
+        for (int p = p0; p < p1; ++p) {
+            const bool ok = valid[p] != 0;
+            const uint8_t mk = mask[p];
+            const bool nw = ok && mk != 0;
+            const bool od = ok && base_mask[p] != 0;
+            if (mode == 0) {
+                if (nw)
+                    list[pos++] = static_cast<uint32_t>(p);
+            } else if (nw != od) {
+                list[pos++] = static_cast<uint32_t>(p) | (od ? 0x80000000u : 0u);
+            }
+            base_mask[p] = mk;
+        }
+        if (threadIdx.x == 0)
+            *count = total;
+        return;
+    }
+    const long long stride = static_cast<long long>(gridDim.x - 1) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n_vec; i += stride)
+        out[i] = mode == 0 ? make_uint4(0u, 0u, 0u, 0u) : base_img[i];
+}
+
+__global__ void k_copy(uint4 *__restrict__ dst, const uint4 *__restrict__ src, long long n_vec)
+{
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_vec;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        dst[i] = src[i];
+}
+
+// ---------------------------------------------------------------------------
+// a6: fused decode + masked reduce (the hot kernel)
+// ---------------------------------------------------------------------------
+// Persistent CTAs, one per SM; the 32 models' decode tables (128 KB) live in
+// shared memory.  Work is a 1-D list of warp tasks (touched block row, tile of
+// 32 listed pixels); a CTA takes WARPS consecutive tasks at a time, each warp
+// decodes its 32 streams (one per lane) 32 scans at a time and reduces them
+// across the warp with redux.sync, adding each scan's total into a per-row
+// shared accumulator; the CTA then adds its rows to the output with one
+// global atomic per nonzero scan sum.
+template <int W>
+__device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint32_t *list,
+                                            uint32_t n, int tile, long long b, uint32_t *acc, int lane,
+                                            DevStatus *st)
+{
+    const uint32_t idx = static_cast<uint32_t>(tile) * 32u + static_cast<uint32_t>(lane);
+    const bool listed = idx < n;
+    const uint32_t e = listed ? __ldg(list + idx) : 0u;
+    const int p = static_cast<int>(e & 0x7FFFFFFFu);
+    const bool neg = (e >> 31) != 0u;
+    Stream S;
+    S.form = kEmpty;
+    S.model = 0;
+    S.shift = 0;
+    S.base = 0;
+    S.c = 0;
+    S.x = 0;
+    S.len = 0;
+    bool ok = listed;
+    if (ok)
+        ok = locate(v, b, p, S.s, S.len, st);
+    if (ok)
+        ok = open_stream(S, W, b, p, st);
+    if (!ok)
+        S.form = kEmpty;
+
+    const unsigned nact = __popc(__ballot_sync(kFull, listed));
+    if (lane == 0) {
+        if (tile == 0)
+            atomicAdd(&st->rows, 1ull);
+        atomicAdd(&st->streams, static_cast<unsigned long long>(nact));
+    }
+
+    const uint32_t *dec = s_dec + S.model * kStates;
+    const bool fast = S.form == kPaired && S.shift == 0 && S.base == 0u;
+    uint32_t over = 0;
+
+    if (W == 1) {
+        // counts fit 16-bit halves: pack scans (2j, 2j+1) into one word; a
+        // leaving pixel contributes 255 - v per half and the warp subtracts
+        // 255 x (number of such lanes) afterwards.
+        const bool packed_src = S.form == kPaired || S.form == kLiteral || S.form == kConstant;
+        const uint32_t flip = (neg && packed_src) ? 0x00FF00FFu : 0u;
+        const uint32_t corr = 255u * static_cast<uint32_t>(__popc(__ballot_sync(kFull, neg && packed_src)));
+        const uint32_t cpk = S.form == kConstant ? (S.c | (S.c << 16)) : 0u;
+        for (int seg = 0; seg < 16; ++seg) {
+            uint32_t pk[16];
+            if (fast) {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    if (jj % 3 == 0 && S.bt.n < 30)
+                        S.bt.refill();
+                    pk[jj] = __byte_perm(tans_step(S, dec), 0u, 0x4342);
+                }
+            } else if (S.form == kPaired) {
+                uint32_t vv[32];
+                paired_segment(S, dec, vv, over);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj)
+                    pk[jj] = vv[2 * jj] | (vv[2 * jj + 1] << 16);
+            } else if (S.form == kLiteral) {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    if (S.bt.n < 16)
+                        S.bt.refill();
+                    const uint32_t a = S.bt.get(8);
+                    const uint32_t c = S.bt.get(8);
+                    pk[jj] = a | (c << 16);
+                }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj)
+                    pk[jj] = cpk;
+            }
+            uint32_t mine = 0;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const uint32_t r = __reduce_add_sync(kFull, pk[jj] ^ flip);
+                if ((lane >> 1) == jj)
+                    mine = r;
+            }
+            mine = ((lane & 1) ? (mine >> 16) : (mine & 0xFFFFu)) - corr;
+            if (mine)
+                atomicAdd(acc + seg * 32 + lane, mine);
+        }
+    } else {
+        const uint32_t sgn = neg ? 0xFFFFFFFFu : 0u;       // v -> (v ^ sgn) - sgn negates
+        for (int seg = 0; seg < 16; ++seg) {
+            uint32_t vv[32];
+            if (S.form == kPaired) {
+                paired_segment(S, dec, vv, over);
+            } else if (S.form == kLiteral) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if (S.bt.n < 16)
+                        S.bt.refill();
+                    vv[i] = S.bt.get(16);
+                }
+            } else {
+                const uint32_t c = S.form == kConstant ? S.c : 0u;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    vv[i] = c;
+            }
+            uint32_t mine = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t r = __reduce_add_sync(kFull, (vv[i] ^ sgn) - sgn);
+                if (lane == i)
+                    mine = r;
+            }
+            if (mine)
+                atomicAdd(acc + seg * 32 + lane, mine);
+        }
+    }
+
+    if (S.form == kPaired) {
+        if (over > (W == 1 ? 0xFFu : 0xFFFFu)) {
+            report(st, kErrValue, b, p);
+        }
+        close_paired(S, b, p, st);
+    } else if (S.form == kSparse) {
+        // sparse: scatter the nonzeros (positions strictly ascending, values nonzero)
+        int prev = -1;
+        bool bad = false;
+        for (uint32_t k = 0; k < S.c; ++k) {
+            if (S.bt.n < 9)
+                S.bt.refill();
+            const int pos = static_cast<int>(S.bt.get(9));
+            if (S.br.n < 16)
+                S.br.refill();
+            const uint32_t val = S.br.get(8 * W);
+            if (pos <= prev || val == 0u) {
+                bad = true;
+                break;
+            }
+            prev = pos;
+            atomicAdd(acc + pos, neg ? 0u - val : val);
+        }
+        if (bad) {
+            report(st, kErrSparse, b, p);
+        } else {
+            const int pad = static_cast<int>(((9u * S.c + 7u) / 8u) * 8u - 9u * S.c);
+            if (pad) {
+                if (S.bt.n < pad)
+                    S.bt.refill();
+                if (S.bt.get(pad) != 0u)
+                    report(st, kErrPad, b, p);
+            }
+        }
+    }
+}
+
+template <int W, int THREADS>
+__global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint32_t *__restrict__ dec_g,
+                                                             const uint32_t *__restrict__ list,
+                                                             const uint32_t *__restrict__ count, int stride,
+                                                             long long rows, void *__restrict__ out,
+                                                             int out_bytes, DevStatus *__restrict__ st)
+{
+    constexpr int WARPS = THREADS / 32;
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *s_dec = smem;
+    uint32_t *s_acc = smem + kModels * kStates;
+    for (int i = threadIdx.x; i < kModels * kStates / 4; i += THREADS)
+        reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
+
+    const uint32_t n = __ldg(count);
+    const long long tiles = (n + 31u) >> 5;
+    const long long total = rows * tiles;
+    const long long ranges = (total + WARPS - 1) / WARPS;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (long long r = blockIdx.x; r < ranges; r += gridDim.x) {
+        const long long t0 = r * WARPS;
+        const long long row0 = t0 / tiles;
+        const long long tl = min(total - 1, t0 + WARPS - 1);
+        const int nslot = static_cast<int>(tl / tiles - row0 + 1);
+        for (int i = threadIdx.x; i < nslot * kScans; i += THREADS)
+            s_acc[i] = 0u;
+        __syncthreads();
+        const long long task = t0 + warp;
+        if (task < total) {
+            const long long row = task / tiles;
+            const int tile = static_cast<int>(task - row * tiles);
+            decode_task<W>(v, s_dec, list, n, tile, row * stride, s_acc + (row - row0) * kScans, lane, st);
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < nslot * kScans; i += THREADS) {
+            const uint32_t val = s_acc[i];
+            if (val) {
+                const long long o = (row0 + i / kScans) * kScans + (i % kScans);
+                if (out_bytes == 4)
+                    atomicAdd(reinterpret_cast<unsigned int *>(out) + o, val);
+                else
+                    atomicAdd(reinterpret_cast<unsigned long long *>(out) + o,
+                              static_cast<unsigned long long>(static_cast<long long>(static_cast<int>(val))));
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a7: block decode into native frames
+// ---------------------------------------------------------------------------
+template <int W>
+__global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_t *__restrict__ dec_g,
+                                                          long long first, long long nblk, void *__restrict__ out,
+                                                          DevStatus *__restrict__ st)
+{
+    using T = typename std::conditional<W == 1, uint8_t, uint16_t>::type;
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *s_dec = smem;
+    for (int i = threadIdx.x; i < kModels * kStates / 4; i += blockDim.x)
+        reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
+    __syncthreads();
+    T *o = reinterpret_cast<T *>(out);
+    const long long total = nblk * v.P;
+    for (long long sid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; sid < total;
+         sid += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long bi = sid / v.P;
+        const int p = static_cast<int>(sid - bi * v.P);
+        const long long b = first + bi;
+        T *dst = o + static_cast<size_t>(bi) * kScans * v.P + p;
+        const size_t P = static_cast<size_t>(v.P);
+        Stream S;
+        S.form = kEmpty;
+        S.model = 0;
+        S.shift = 0;
+        S.base = 0;
+        S.c = 0;
+        S.x = 0;
+        S.len = 0;
+        bool ok = v.valid[p] != 0;
+        if (ok)
+            ok = locate(v, b, p, S.s, S.len, st);
+        if (ok)
+            ok = open_stream(S, W, b, p, st);
+        if (!ok)
+            S.form = kEmpty;
+        if (S.form == kPaired) {
+            const uint32_t *dec = s_dec + S.model * kStates;
+            uint32_t over = 0;
+            for (int seg = 0; seg < 16; ++seg) {
+                uint32_t vv[32];
+                paired_segment(S, dec, vv, over);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    dst[(seg * 32 + i) * P] = static_cast<T>(vv[i]);
+            }
+            if (over > (W == 1 ? 0xFFu : 0xFFFFu))
+                report(st, kErrValue, b, p);
+            close_paired(S, b, p, st);
+        } else if (S.form == kLiteral) {
+            for (int i = 0; i < kScans; ++i) {
+                if (S.bt.n < 16)
+                    S.bt.refill();
+                dst[i * P] = static_cast<T>(S.bt.get(8 * W));
+            }
+        } else if (S.form == kSparse) {
+            int prev = -1;
+            bool bad = false;
+            for (uint32_t k = 0; k < S.c; ++k) {
+                if (S.bt.n < 9)
+                    S.bt.refill();
+                const int pos = static_cast<int>(S.bt.get(9));
+                if (S.br.n < 16)
+                    S.br.refill();
+                const uint32_t val = S.br.get(8 * W);
+                if (pos <= prev || val == 0u) {
+                    bad = true;
+                    break;
+                }
+                for (int i = prev + 1; i < pos; ++i)
+                    dst[i * P] = 0;
+                dst[pos * P] = static_cast<T>(val);
+                prev = pos;
+            }
+            for (int i = prev + 1; i < kScans; ++i)
+                dst[i * P] = 0;
+            if (bad) {
+                report(st, kErrSparse, b, p);
+            } else {
+                const int pad = static_cast<int>(((9u * S.c + 7u) / 8u) * 8u - 9u * S.c);
+                if (pad) {
+                    if (S.bt.n < pad)
+                        S.bt.refill();
+                    if (S.bt.get(pad) != 0u)
+                        report(st, kErrPad, b, p);
+                }
+            }
+        } else {
+            const T c = static_cast<T>(S.form == kConstant ? S.c : 0u);
+            for (int i = 0; i < kScans; ++i)
+                dst[i * P] = c;
+        }
+    }
+}
+
+int sm_count()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0)
+            n = 1;
+    }
+    return n;
+}
+
+constexpr size_t kTableBytes = static_cast<size_t>(kModels) * kStates * sizeof(uint32_t);
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_generate(void *out, int bits, uint64_t seed, int64_t scan0, int64_t n_scans, int P,
+                            const uint32_t *pclass, const uint32_t *desc, const uint64_t *thr, cudaStream_t st)
+{
+    if (n_scans <= 0 || P <= 0)
+        return cudaSuccess;
+    dim3 block(256);
+    dim3 grid((P + 255) / 256, static_cast<unsigned>(n_scans < 4096 ? n_scans : 4096));
+    const uint4 *d = reinterpret_cast<const uint4 *>(desc);
+    if (bits == 8)
+        k_generate<uint8_t><<<grid, block, 0, st>>>(static_cast<uint8_t *>(out), seed, scan0, n_scans, P, pclass,
+                                                    d, thr, 0xFFu);
+    else
+        k_generate<uint16_t><<<grid, block, 0, st>>>(static_cast<uint16_t *>(out), seed, scan0, n_scans, P,
+                                                     pclass, d, thr, 0xFFFFu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_enc_streams(const void *counts, int w, int P, int nblk, Tables tb, uint4 *desc, uint32_t *slots,
+                               unsigned long long *stats, cudaStream_t st)
+{
+    const long long total = static_cast<long long>(nblk) * P;
+    const unsigned grid = static_cast<unsigned>((total + kEncThreads - 1) / kEncThreads);
+    if (w == 1)
+        k_enc_streams<uint8_t><<<grid, kEncThreads, 0, st>>>(static_cast<const uint8_t *>(counts), P, nblk, tb,
+                                                             desc, slots, stats);
+    else
+        k_enc_streams<uint16_t><<<grid, kEncThreads, 0, st>>>(static_cast<const uint16_t *>(counts), P, nblk, tb,
+                                                              desc, slots, stats);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_enc_layout(uint4 *desc, int P, int G, int nblk, uint32_t *groups, uint32_t *blk_len,
+                              cudaStream_t st)
+{
+    k_enc_layout<<<nblk, kLayoutThreads, 0, st>>>(desc, P, G, groups, blk_len);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const uint4 *desc,
+                               const uint32_t *slots, const unsigned long long *blk_dst, cudaStream_t st)
+{
+    const long long total = static_cast<long long>(nblk) * P;
+    const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+    if (w == 1)
+        k_enc_compact<uint8_t><<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(counts), P, nblk, desc, slots,
+                                                     blk_dst);
+    else
+        k_enc_compact<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(counts), P, nblk, desc,
+                                                      slots, blk_dst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, uint8_t *base_mask, int P, int mode,
+                        uint32_t *list, uint32_t *count, void *out, const void *base_img, long long n_elems,
+                        int out_bytes, cudaStream_t st)
+{
+    const long long n_vec = n_elems * out_bytes / 16;
+    int fill = static_cast<int>((n_vec + kPlanThreads - 1) / kPlanThreads);
+    fill = fill < 1 ? 1 : (fill > 4 * sm_count() ? 4 * sm_count() : fill);
+    k_plan<<<1 + fill, kPlanThreads, 0, st>>>(mask, valid, base_mask, P, mode, list, count,
+                                              static_cast<uint4 *>(out), static_cast<const uint4 *>(base_img),
+                                              n_vec);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy(void *dst, const void *src, size_t bytes, cudaStream_t st)
+{
+    const long long n_vec = static_cast<long long>(bytes / 16);
+    int grid = static_cast<int>((n_vec + 255) / 256);
+    grid = grid < 1 ? 1 : (grid > 4 * sm_count() ? 4 * sm_count() : grid);
+    k_copy<<<grid, 256, 0, st>>>(static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), n_vec);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride,
+                                 long long rows, void *out, int out_bytes, DevStatus *status, int n_sm,
+                                 cudaStream_t st)
+{
+    if (v.w == 1) {
+        constexpr int TH = 1024;
+        const size_t smem = kTableBytes + static_cast<size_t>(TH / 32) * kScans * sizeof(uint32_t);
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(k_decode_reduce<1, TH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+            attr = true;
+        }
+        k_decode_reduce<1, TH><<<n_sm, TH, smem, st>>>(v, tb.dec, list, count, stride, rows, out, out_bytes,
+                                                       status);
+    } else {
+        constexpr int TH = 512;
+        const size_t smem = kTableBytes + static_cast<size_t>(TH / 32) * kScans * sizeof(uint32_t);
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(k_decode_reduce<2, TH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+            attr = true;
+        }
+        k_decode_reduce<2, TH><<<n_sm, TH, smem, st>>>(v, tb.dec, list, count, stride, rows, out, out_bytes,
+                                                       status);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,
+                                 cudaStream_t st)
+{
+    const size_t smem = kTableBytes;
+    const int grid = sm_count();
+    if (v.w == 1) {
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(k_decode_blocks<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+            attr = true;
+        }
+        k_decode_blocks<1><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
+    } else {
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(k_decode_blocks<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+            attr = true;
+        }
+        k_decode_blocks<2><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace qem

@@ -1,0 +1,111 @@
+// qem_internal.h -- shared declarations of libqem's host code and kernels.
+//
+// Bitstream: qem-pair-v1 (page "Paired-count resident layout", "Operation
+// pipeline" step 2 and "Contract"; the bit-level choices are the library's
+// own written spec, sections S1-S7, cited as "spec Sn").
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qem.h"
+
+namespace qem {
+
+constexpr int kScans = 512;        // scans per block (page: complete 512-scan blocks)
+constexpr int kPairs = 256;        // consecutive count pairs per stream
+constexpr int kStates = 1024;      // tANS states (page: 1024-state table)
+constexpr int kModels = 32;        // Poisson pair models (page: 32)
+constexpr int kGroupWords = 17;    // 1 x u32 base + 32 x u16 relative ends (spec S1)
+constexpr int kSlotWords = 82;     // per-stream tANS scratch: ceil((10 + 256*10)/32) + 1 words
+constexpr int kArenaPad = 64;      // zero bytes after the last block of an arena
+
+enum Form : int { kEmpty = 0, kConstant = 1, kSparse = 2, kPaired = 3, kLiteral = 4 };
+
+// device status flags (spec S7); any nonzero flag means "malformed"
+enum : uint32_t {
+    kErrReserved = 1u << 0,
+    kErrForm = 1u << 1,
+    kErrFields = 1u << 2,
+    kErrLength = 1u << 3,
+    kErrSparse = 1u << 4,
+    kErrConstant = 1u << 5,
+    kErrState = 1u << 6,
+    kErrPad = 1u << 7,
+    kErrOffsets = 1u << 8,
+    kErrValue = 1u << 9,
+};
+
+struct DevStatus {
+    uint32_t flags;
+    uint32_t first_block;
+    uint32_t first_pixel;
+    uint32_t have_first;
+    unsigned long long rows;      // touched block rows decoded by masked sums
+    unsigned long long streams;   // streams decoded by masked sums
+};
+
+// Device-resident model tables.
+//  dec[m][slot]   : bits 0-9 newbase, 10-13 nb, byte 2 = hi_a, byte 3 = hi_b
+//  enc_sym[m][s]  : bits 0-10 f, 11-21 cum (start of s in enc_slot), 22-25 k0 = 10 - floor(log2 f)
+//  enc_slot[m][i] : slots of each symbol in ascending order, grouped by symbol
+//  cost[m][v], amax[m] : selection costs and box sizes (spec S4)
+struct Tables {
+    const uint32_t *dec;
+    const uint32_t *enc_sym;
+    const uint16_t *enc_slot;
+    const uint32_t *cost;
+    const uint32_t *amax;
+};
+
+struct HostTables {
+    uint16_t freq[kModels][256];
+    uint8_t amax[kModels];
+    uint32_t cost[kModels][16];
+    uint32_t dec[kModels][kStates];
+    uint32_t enc_sym[kModels][256];
+    uint16_t enc_slot[kModels][kStates];
+};
+
+// What the query kernels read of a resident.
+struct View {
+    const uint32_t *groups;               // [B][G][17]
+    const unsigned long long *blk_ptr;    // [B] device address of each block's payload
+    const uint32_t *blk_len;              // [B] payload bytes of each block
+    const uint8_t *valid;                 // [P]
+    int P;
+    int G;
+    int w;                                // bytes per count (1 or 2)
+    long long B;
+};
+
+const HostTables &host_tables();          // built once per process (tables.cu)
+
+// ---- kernel launchers (kernels.cu); all stream-ordered, return cudaError_t ----
+cudaError_t launch_generate(void *out, int bits, uint64_t seed, int64_t scan0, int64_t n_scans,
+                            int P, const uint32_t *pclass, const uint32_t *desc,
+                            const uint64_t *thr, cudaStream_t st);
+
+cudaError_t launch_enc_streams(const void *counts, int w, int P, int nblk, Tables tb,
+                               uint4 *desc, uint32_t *slots, unsigned long long *stats,
+                               cudaStream_t st);
+cudaError_t launch_enc_layout(uint4 *desc, int P, int G, int nblk, uint32_t *groups,
+                              uint32_t *blk_len, cudaStream_t st);
+cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const uint4 *desc,
+                               const uint32_t *slots, const unsigned long long *blk_dst,
+                               cudaStream_t st);
+
+// plan: builds the signed pixel list (CTA 0) and initialises the output rows
+// (other CTAs): mode 0 = full query (out = 0), 1 = delta (out = baseline image)
+cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, uint8_t *base_mask, int P,
+                        int mode, uint32_t *list, uint32_t *count, void *out,
+                        const void *base_img, long long n_elems, int out_bytes,
+                        cudaStream_t st);
+cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count,
+                                 int stride, long long rows, void *out, int out_bytes,
+                                 DevStatus *status, int n_sm, cudaStream_t st);
+cudaError_t launch_copy(void *dst, const void *src, size_t bytes, cudaStream_t st);
+cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out,
+                                 DevStatus *status, cudaStream_t st);
+
+}  // namespace qem
