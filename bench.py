@@ -1,0 +1,456 @@
+"""Benchmark of the paired-count resident on B200.
+
+Workload (default): the 512x512-scan, 192x192-pixel uint8 acquisition
+(9.66 GB raw, counter-based synthetic Poisson counts: bright-field disk r=30
+with lambda=3, lambda=0.01 outside), generated and encoded on the device.
+One step is the query schedule of that workload through the C ABI:
+bright-field and annular (40<=r<=90) masked sums at block_stride 1, 4 and 16,
+then a 65-query drag (a full r=30 disk query followed by 64 one-pixel-shift
+delta queries).  `value` is masked-sum queries per second over all ranks
+with the resident already in HBM; `e2e` repeats the steps with every mask
+copied in from pinned host memory and every image read back to pinned host
+memory inside the timed region.
+
+Each rank holds its own resident and runs the same schedule (independent
+acquisitions, weak scaling, no data-path collective).
+
+--impl reference times the CPU oracle (plain C, test infrastructure) on a
+bounded sample of the same workload and reports the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "masked_sum queries/s and raw-equivalent GB/s decoded at 512x512x192x192 vs HBM roofline"
+UNIT = "queries/s"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def schedule(w: W.Workload):
+    """[(label, mask uint8[P], stride, delta)] for one step."""
+    q = []
+    for k in w.strides:
+        for name in ("bf", "adf"):
+            q.append((f"{name}_k{k}", w.masks[name], k, False))
+    if w.drag:
+        q.append(("drag_full", w.drag[0], 1, False))
+        for t in range(1, len(w.drag)):
+            q.append(("drag_delta", w.drag[t], 1, True))
+    return q
+
+
+def stream_lengths(res, w):
+    """Encoded extent of every stream, [B][P] (from the exported group tables)."""
+    B, P = w.n_blocks, w.n_pixels
+    lens = np.zeros((B, P), np.uint32)
+    for b in range(B):
+        g, _ = res.export_block(b)
+        ends = np.stack([(g[:, 1 + j // 2] >> (16 * (j & 1))) & 0xFFFF for j in range(32)], axis=1)
+        ends = ends.astype(np.int64)
+        starts = np.concatenate([np.zeros((ends.shape[0], 1), np.int64), ends[:, :-1]], axis=1)
+        lens[b] = (ends - starts).reshape(-1)[:P]
+    return lens
+
+
+def algorithmic_bytes(lens, w, sched, out_bits):
+    """Per query: encoded bytes of the listed streams in the touched blocks + 2 B offset per stream +
+    4 B group base per touched group + the image written + the 4 B list entries."""
+    out = []
+    prev = None
+    for label, m, k, delta in sched:
+        sel = m.astype(bool)
+        if delta and prev is not None:
+            lst = sel ^ prev
+        else:
+            lst = sel
+        prev = sel
+        pix = np.nonzero(lst)[0]
+        rows = list(range(0, w.n_blocks, k))
+        enc = int(lens[rows][:, pix].sum(dtype=np.int64))
+        groups = len(np.unique(pix // 32)) * len(rows)
+        img = len(rows) * 512 * out_bits // 8
+        raw = pix.size * 512 * len(rows) * (w.dtype_bits // 8)
+        out.append(dict(label=label, enc=enc, streams=pix.size * len(rows), bytes=enc + 2 * pix.size * len(rows)
+                        + 4 * groups + img + 4 * pix.size, raw=raw))
+    return out
+
+
+class Clocks:
+    """nvidia-smi sampler (every 200 ms) around the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(parts)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def build_resident(w, dev, torch, V, stream=None):
+    """Generate the workload's counts on the device and encode them (chunked for large ones)."""
+    spec = w.counter
+    pc = torch.from_numpy(spec.pixel_class.astype(np.int32)).to(dev)
+    cd = torch.from_numpy(spec.class_desc.astype(np.int32)).to(dev)
+    th = torch.from_numpy(spec.thresholds.view(np.int64)).to(dev)
+    dt = torch.uint8 if w.dtype_bits == 8 else torch.uint16
+    raw_bytes = w.raw_bytes
+    chunk_blocks = w.n_blocks if raw_bytes <= (24 << 30) else 1
+    buf = torch.empty((chunk_blocks * 512, w.n_pixels), dtype=dt, device=dev)
+    res = V.Resident.create((w.scan_rows, w.scan_cols), (w.det_rows, w.det_cols), w.dtype_bits)
+    t_enc = 0.0
+    for b0 in range(0, w.n_blocks, chunk_blocks):
+        nb = min(chunk_blocks, w.n_blocks - b0)
+        V.generate_counts(buf, w.dtype_bits, spec.seed, b0 * 512, nb * 512, w.n_pixels, pc, cd, th)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        res.append(buf, nb)
+        e1.record()
+        torch.cuda.synchronize()
+        t_enc += e0.elapsed_time(e1) / 1e3
+    return res, buf, t_enc
+
+
+def cpu_baseline(w, sample_blocks=4):
+    """The oracle as it stands, on the host cores: BF and ADF k=1 queries over a sample of blocks,
+    scaled to the full acquisition."""
+    import oracle as O
+
+    blocks = list(range(0, w.n_blocks, max(1, w.n_blocks // sample_blocks)))[:sample_blocks]
+    counts = [w.block_counts(b) for b in blocks]
+    enc = O.Encoded(w.n_pixels, w.dtype_bits)
+    for c in counts:
+        g, p = O.encode_block(c, w.dtype_bits)
+        enc.groups.append(g)
+        enc.payloads.append(p)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        for name in ("bf", "adf"):
+            O.resident_masked_sum(enc, w.masks[name], None, 1, threads=threads)
+            n += 1
+        if time.perf_counter() - t0 > 10.0:
+            break
+    dt = (time.perf_counter() - t0) / n
+    full = dt * w.n_blocks / len(blocks)
+    return {"value": 1.0 / full, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"bf/adf k=1 queries over {len(blocks)} of {w.n_blocks} blocks (host-regenerated), "
+                      f"{n} queries in {dt * n:.1f} s, scaled to all blocks"}
+
+
+def run_reference(args, rank, world):
+    import oracle as O
+
+    if rank != 0:
+        return
+    w = W.workload(args.config)
+    sample = 2
+    blocks = [0, w.n_blocks // 2][:sample]
+    enc = O.Encoded(w.n_pixels, w.dtype_bits)
+    for b in blocks:
+        g, p = O.encode_block(w.block_counts(b), w.dtype_bits)
+        enc.groups.append(g)
+        enc.payloads.append(p)
+    sched = [(l, m, 1, d) for (l, m, k, d) in schedule(w)]        # every query over the sampled blocks
+    threads = os.cpu_count() or 1
+
+    def step():
+        prev = None
+        img = None
+        for label, m, k, delta in sched:
+            if delta and prev is not None:
+                img = O.resident_delta(enc, img, prev, m, None, 1, threads=threads)
+            else:
+                img = O.resident_masked_sum(enc, m, None, 1, threads=threads)
+            prev = m
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    step_full = dt * w.n_blocks / len(blocks)      # the schedule's k=1 cost, scaled to all blocks
+    value = len(sched) / step_full
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_full * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8" if w.dtype_bits == 8 else "u16",
+            "data": "synthetic",
+            "config": {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
+                                   f"uint{w.dtype_bits}", "queries_per_step": len(sched)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{len(sched)} queries (all at block_stride 1) over blocks {blocks} of "
+                                       f"{w.n_blocks}, scaled to all blocks"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="c4")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import virtual_imaging_b200 as V
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = W.workload(args.config)
+    res, buf, _ = build_resident(w, dev, torch, V)
+    # a second, warm encode of the same counts for the encode figure (chunked workloads keep the first)
+    enc_s = None
+    if buf.shape[0] == w.n_scans:
+        res2 = V.Resident.create((w.scan_rows, w.scan_cols), (w.det_rows, w.det_cols), w.dtype_bits)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        res2.append(buf, w.n_blocks)
+        e1.record()
+        torch.cuda.synchronize()
+        enc_s = e0.elapsed_time(e1) / 1e3
+        res2.free()
+    # block decode leg (16 blocks)
+    nd = min(16, w.n_blocks)
+    frames = torch.empty((nd * 512, w.n_pixels), dtype=buf.dtype, device=dev)
+    res.decode_blocks(0, nd, out=frames)
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record()
+    res.decode_blocks(0, nd, out=frames, wait=False)
+    d1.record()
+    torch.cuda.synchronize()
+    dec_s = d0.elapsed_time(d1) / 1e3
+    res.finish()
+    ok_frames = bool(torch.equal(frames, buf[: nd * 512])) if buf.shape[0] >= nd * 512 else None
+    del frames
+    del buf
+    torch.cuda.empty_cache()
+
+    info = res.info()
+    out_bits = info["out_bits_auto"]
+    sched = schedule(w)
+    masks = [torch.from_numpy(m.astype(np.uint8)).to(dev) for (_, m, _, _) in sched]
+    outs = {}
+    for label, m, k, d in sched:
+        rows = -(-w.n_blocks // k)
+        outs.setdefault(k, torch.empty((rows, 512), dtype=V.out_dtype(out_bits), device=dev))
+
+    def step(ms=masks):
+        for (label, m, k, delta), md in zip(sched, ms):
+            fn = res.masked_sum_delta if delta else res.masked_sum
+            fn(md, block_stride=k, out=outs[k], wait=False)
+
+    for _ in range(args.warmup):
+        step()
+    res.finish()
+    torch.cuda.synchronize()
+    res.profile(True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    res.finish()
+    t = e0.elapsed_time(e1) / 1e3
+    prof = res.profile_read()
+    res.profile(False)
+    if world > 1:
+        tt = torch.tensor([t], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+
+    # end to end: masks from pinned host memory in, images to pinned host memory out
+    host_masks = [torch.from_numpy(m.astype(np.uint8)).pin_memory() for (_, m, _, _) in sched]
+    dev_masks = [torch.empty_like(h, device=dev) for h in host_masks]
+    host_imgs = [torch.empty(tuple(outs[k].shape), dtype=outs[k].dtype).pin_memory() for (_, _, k, _) in sched]
+    h2d = sum(h.numel() for h in host_masks)
+    d2h = sum(h.numel() * h.element_size() for h in host_imgs)
+
+    def e2e_step():
+        for (label, m, k, delta), hm, dm, hi in zip(sched, host_masks, dev_masks, host_imgs):
+            dm.copy_(hm, non_blocking=True)
+            fn = res.masked_sum_delta if delta else res.masked_sum
+            fn(dm, block_stride=k, out=outs[k], wait=False)
+            hi.copy_(outs[k], non_blocking=True)
+
+    e2e_step()
+    res.finish()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    res.finish()
+    te = f0.elapsed_time(f1) / 1e3
+    if world > 1:
+        tt = torch.tensor([te], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        te = float(tt.item())
+
+    # per-query breakdown (separate, untimed for `value`)
+    lens = stream_lengths(res, w)
+    ab = algorithmic_bytes(lens, w, sched, out_bits)
+    per_query = {}
+    for (label, m, k, delta), md, a in zip(sched, masks, ab):
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn = res.masked_sum_delta if delta else res.masked_sum
+        q0.record()
+        fn(md, block_stride=k, out=outs[k], wait=False)
+        q1.record()
+        torch.cuda.synchronize()
+        d = per_query.setdefault(label, {"ms": [], "enc_bytes": a["enc"], "raw_bytes": a["raw"]})
+        d["ms"].append(q0.elapsed_time(q1))
+    res.finish()
+    for d in per_query.values():
+        d["ms"] = statistics.median(d["ms"])
+        d["raw_equiv_gbs"] = d["raw_bytes"] / (d["ms"] / 1e3) / 1e9
+        d["enc_gbs"] = d["enc_bytes"] / (d["ms"] / 1e3) / 1e9
+
+    hbm, peak_kind = peaks()
+    n_dec, ms_dec = prof["decode_reduce"]
+    bytes_step = sum(a["bytes"] for a in ab)
+    raw_step = sum(a["raw"] for a in ab)
+    achieved = bytes_step * args.steps / (ms_dec / 1e3) / 1e9 if ms_dec > 0 else None
+    launches = sum(prof[k][0] for k in ("plan", "decode_reduce", "finalize"))
+    clocks = clk.summary()
+
+    nq = len(sched)
+    line = {
+        "metric": METRIC, "value": world * nq * args.steps / t, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8" if w.dtype_bits == 8 else "u16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
+                               f"uint{w.dtype_bits}, counter-based Poisson (BF r=30 lambda=3, outside 0.01)",
+                   "queries_per_step": nq, "schedule": "bf/adf at block_stride 1,4,16 + drag: 1 full + 64 deltas",
+                   "parallelism": f"{world} independent residents (one per GPU)",
+                   "l2": f"inputs larger than L2: {bytes_step / 1e9:.2f} GB of encoded streams read per step",
+                   "resident_bytes": info["payload_bytes"] + info["group_bytes"], "raw_bytes": w.raw_bytes},
+        "raw_equiv_gbs": world * raw_step * args.steps / t / 1e9,
+        "e2e": {"value": world * nq * args.steps / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": (achieved / hbm) if achieved else None, "traffic": None,
+                     "kernel": "k_decode_reduce", "peak_kind": peak_kind,
+                     "avg_launch_ms": ms_dec / max(1, n_dec), "launches": n_dec,
+                     "algorithmic_bytes_per_launch": bytes_step * args.steps / max(1, n_dec)},
+        "queries": {k: {"ms": round(v["ms"], 4), "raw_equiv_gbs": round(v["raw_equiv_gbs"], 1),
+                        "enc_gbs": round(v["enc_gbs"], 1), "hbm_frac_enc": round(v["enc_gbs"] / hbm, 4)}
+                    for k, v in per_query.items()},
+        "kernels_ms_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[0]},
+        "encode": {"gbs_raw": (w.raw_bytes / enc_s / 1e9) if enc_s else None, "s": enc_s,
+                   "hbm_frac": ((w.raw_bytes + info["payload_bytes"] + info["group_bytes"]) / enc_s / 1e9 / hbm)
+                   if enc_s else None},
+        "decode_blocks": {"blocks": nd, "s": dec_s, "gcounts_per_s": nd * 512 * w.n_pixels / dec_s / 1e9,
+                          "exact": ok_frames},
+        "resident": {"payload_bytes": info["payload_bytes"], "forms": info["form_count"],
+                     "bits_per_count": 8 * info["payload_bytes"] / (w.n_scans * w.n_pixels)},
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    res.free()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
