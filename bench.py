@@ -207,38 +207,39 @@ def cpu_baseline(w, sample_blocks=4):
 
 
 def run_reference(args, rank, world):
+    """The oracle timed on the host cores on a bounded sample (2 blocks) of the same workload and schedule:
+    every query of the step runs over the sampled blocks, and its time per block is scaled by the number
+    of blocks the query touches in the full acquisition (ceil(B/k))."""
     import oracle as O
 
     if rank != 0:
         return
     w = W.workload(args.config)
-    sample = 2
-    blocks = [0, w.n_blocks // 2][:sample]
+    blocks = [0, w.n_blocks // 2]
     enc = O.Encoded(w.n_pixels, w.dtype_bits)
     for b in blocks:
         g, p = O.encode_block(w.block_counts(b), w.dtype_bits)
         enc.groups.append(g)
         enc.payloads.append(p)
-    sched = [(l, m, 1, d) for (l, m, k, d) in schedule(w)]        # every query over the sampled blocks
+    sched = schedule(w)
     threads = os.cpu_count() or 1
 
     def step():
-        prev = None
-        img = None
+        prev = img = None
+        scaled = 0.0
         for label, m, k, delta in sched:
+            t0 = time.perf_counter()
             if delta and prev is not None:
                 img = O.resident_delta(enc, img, prev, m, None, 1, threads=threads)
             else:
                 img = O.resident_masked_sum(enc, m, None, 1, threads=threads)
+            scaled += (time.perf_counter() - t0) / len(blocks) * math.ceil(w.n_blocks / k)
             prev = m
+        return scaled
 
     for _ in range(args.warmup):
         step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    step_full = dt * w.n_blocks / len(blocks)      # the schedule's k=1 cost, scaled to all blocks
+    step_full = sum(step() for _ in range(args.steps)) / args.steps
     value = len(sched) / step_full
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_full * 1e3, "higher_is_better": True,
@@ -247,10 +248,28 @@ def run_reference(args, rank, world):
             "config": {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
                                    f"uint{w.dtype_bits}", "queries_per_step": len(sched)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": f"{len(sched)} queries (all at block_stride 1) over blocks {blocks} of "
-                                       f"{w.n_blocks}, scaled to all blocks"},
+                             "sample": f"each of the {len(sched)} queries of a step timed over blocks {blocks} of "
+                                       f"{w.n_blocks} and scaled to the ceil(B/k) blocks it touches"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_profile_case(dev, torch, V):
+    """Small bounded case for ncu: build the default resident, then a few bright-field / annular
+    block_stride-1 queries (the kernels ncu captures are the k_decode_reduce launches)."""
+    w = W.workload("c4")
+    res, buf, t_enc = build_resident(w, dev, torch, V)
+    del buf
+    torch.cuda.empty_cache()
+    out = torch.empty((w.n_blocks, 512), dtype=V.out_dtype(32), device=dev)
+    bf = torch.from_numpy(w.masks["bf"]).to(dev)
+    adf = torch.from_numpy(w.masks["adf"]).to(dev)
+    res.profile(True)
+    for m in (bf, adf, bf, adf):
+        res.masked_sum(m, out=out)
+    p = res.profile_read()
+    print(json.dumps({"encode_s": t_enc, "kernels": p}), flush=True)
+    res.free()
 
 
 def main():
@@ -261,6 +280,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="c4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true", help="bounded case for ncu captures")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -281,6 +301,9 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
+    if args.profile:
+        run_profile_case(dev, torch, V)
+        return
     w = W.workload(args.config)
     res, buf, _ = build_resident(w, dev, torch, V)
     # a second, warm encode of the same counts for the encode figure (chunked workloads keep the first)
