@@ -173,6 +173,38 @@ int qem_profile_read(qem_resident *res, qem_profile_t *out);
  * pipeline": the resident owns its arrays).  NULL is ignored. */
 void qem_free(qem_resident *res);
 
+/* ---- masked sum that allocates nothing ---- */
+
+/* Largest detector (pixels) qem_masked_sum_noalloc accepts. */
+#define QEM_NOALLOC_MAX_PIXELS 131072
+
+/* Masked sum for callers that cannot allocate device memory while they query:
+ * for example a render or acquisition thread that must never block on the
+ * CUDA allocator (cudaMalloc can synchronise the device and stall it), code
+ * that runs under an external memory budget which forbids new allocations
+ * once set-up is over, or a host application whose allocator is owned by
+ * another framework.  The source pages have no counterpart to this call.
+ *
+ * Same result as qem_masked_sum (same d_mask, block_stride, out_bits and
+ * d_out rules; d_out is caller-owned) but this call performs no cudaMalloc,
+ * cudaFree or other allocating routine.  Its working memory (the listed
+ * pixels, their count and the error status, ~0.5 MB) is one fixed array in
+ * the library's device globals, held by every GPU that loads the library
+ * until the process exits.  Consequences:
+ *  - the detector may have at most QEM_NOALLOC_MAX_PIXELS pixels, otherwise
+ *    QEM_ERR_ARG is returned and nothing runs;
+ *  - all calls share that array: calls whose work overlaps on the GPU (other
+ *    streams, other threads) race and give wrong results; serialise them;
+ *  - the first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture;
+ *  - the call waits for its own work on `stream` and returns
+ *    QEM_ERR_MALFORMED if a decoded stream failed a check;
+ *  - it neither reads nor updates the per-stride delta baselines.
+ * The resident must live on the current device and be complete. */
+int qem_masked_sum_noalloc(qem_resident *res, const uint8_t *d_mask, int32_t block_stride,
+                           int32_t out_bits, void *d_out, void *stream);
+
 /* ---- encoded form, host side (export for inspection/saving, import) ---- */
 
 /* Payload length of block b in bytes. */

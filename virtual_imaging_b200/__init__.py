@@ -30,7 +30,7 @@ FORMS = ("empty", "constant", "sparse", "paired", "literal")
 EXPORTS = ("qem_abi", "qem_status_string", "qem_create", "qem_encode", "qem_encode_append", "qem_masked_sum",
            "qem_masked_sum_delta", "qem_decode_blocks", "qem_finish", "qem_info", "qem_query_counters",
            "qem_profile", "qem_profile_read", "qem_free", "qem_block_bytes", "qem_export_block", "qem_import",
-           "qem_model_tables", "qem_generate_counts")
+           "qem_model_tables", "qem_generate_counts", "qem_masked_sum_noalloc")
 
 
 class QemError(RuntimeError):
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
         "qem_import": ([i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, pp], ctypes.c_int),
         "qem_model_tables": ([vp, vp, vp], ctypes.c_int),
         "qem_generate_counts": ([vp, i32, u64, i64, i64, i32, vp, vp, vp, vp], ctypes.c_int),
+        "qem_masked_sum_noalloc": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -219,6 +220,15 @@ class Resident:
                          out: torch.Tensor | None = None, wait: bool = True, stream=None) -> torch.Tensor:
         return self._query(lib().qem_masked_sum_delta, "qem_masked_sum_delta", mask, block_stride, out_bits,
                            out, wait, stream)
+
+    def masked_sum_noalloc(self, mask: torch.Tensor, out: torch.Tensor, block_stride: int = 1,
+                           out_bits: int = 0, stream=None) -> torch.Tensor:
+        """Masked sum that allocates no device memory (qem_masked_sum_noalloc): for callers that
+        must not allocate while querying.  `out` must be preallocated ([ceil(B/k)][512] of the
+        chosen width); calls that overlap on the GPU race on the library's fixed working memory."""
+        _check(lib().qem_masked_sum_noalloc(self._h, _dev_ptr(mask), block_stride, out_bits, _dev_ptr(out),
+                                            _stream(stream)), "qem_masked_sum_noalloc")
+        return out
 
     def decode_blocks(self, first: int, n: int, out: torch.Tensor | None = None, wait: bool = True,
                       stream=None) -> torch.Tensor:

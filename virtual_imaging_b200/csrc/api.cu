@@ -789,3 +789,22 @@ int qem_generate_counts(void *d_out, int32_t dtype_bits, uint64_t seed, int64_t 
 }
 
 }  // extern "C"
+
+// Read-only view of a resident for the allocation-free masked sum (noalloc.cu).
+namespace qem {
+int resident_query_view(const qem_resident *r, ResidentQuery *q)
+{
+    if (!r || !q)
+        return QEM_ERR_ARG;
+    q->view = r->view();
+    q->tables = r->tables();
+    q->P = r->P;
+    q->B = r->B;
+    q->complete = r->B_done == r->B;
+    q->out_bits_auto = r->out_bits_auto;
+    q->n_sm = r->n_sm;
+    q->device = r->device;
+    q->valid = r->d_valid;
+    return QEM_OK;
+}
+}  // namespace qem

@@ -81,6 +81,20 @@ struct View {
 
 const HostTables &host_tables();          // built once per process (tables.cu)
 
+// What the allocation-free masked sum needs from a resident (api.cu).
+struct ResidentQuery {
+    View view;
+    Tables tables;
+    int P;
+    long long B;
+    bool complete;
+    int out_bits_auto;
+    int n_sm;
+    int device;
+    const uint8_t *valid;
+};
+int resident_query_view(const qem_resident *r, ResidentQuery *q);
+
 // ---- kernel launchers (kernels.cu); all stream-ordered, return cudaError_t ----
 cudaError_t launch_generate(void *out, int bits, uint64_t seed, int64_t scan0, int64_t n_scans,
                             int P, const uint32_t *pclass, const uint32_t *desc,
