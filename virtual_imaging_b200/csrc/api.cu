@@ -63,6 +63,8 @@ struct qem_resident {
     std::vector<Arena> arenas;
 
     uint32_t *d_dec = nullptr, *d_enc_sym = nullptr, *d_cost = nullptr, *d_amax = nullptr;
+    uint16_t *d_skip = nullptr;
+    uint32_t skip_models = 0;
     uint16_t *d_enc_slot = nullptr;
 
     uint4 *d_desc = nullptr;
@@ -86,7 +88,7 @@ struct qem_resident {
     std::vector<ProfEvent> events;
     qem_profile_t prof_acc{};
 
-    Tables tables() const { return Tables{d_dec, d_enc_sym, d_enc_slot, d_cost, d_amax}; }
+    Tables tables() const { return Tables{d_dec, d_enc_sym, d_enc_slot, d_cost, d_amax, d_skip, skip_models}; }
     View view() const { return View{d_groups, d_blk_ptr, d_blk_len, d_valid, P, G, w, B}; }
 };
 
@@ -182,6 +184,7 @@ void release(qem_resident *r)
     cudaFree(r->d_enc_slot);
     cudaFree(r->d_cost);
     cudaFree(r->d_amax);
+    cudaFree(r->d_skip);
     cudaFree(r->d_desc);
     cudaFree(r->d_slots);
     cudaFree(r->d_stats);
@@ -253,7 +256,7 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
         (rc = dalloc(&r->d_blk_ptr, size_t(r->B) * 8)) || (rc = dalloc(&r->d_blk_len, size_t(r->B) * 4)) ||
         (rc = dalloc(&r->d_dec, sizeof(T.dec))) || (rc = dalloc(&r->d_enc_sym, sizeof(T.enc_sym))) ||
         (rc = dalloc(&r->d_enc_slot, sizeof(T.enc_slot))) || (rc = dalloc(&r->d_cost, sizeof(T.cost))) ||
-        (rc = dalloc(&r->d_amax, kModels * 4)) || (rc = dalloc(&r->d_stats, (5 + kModels) * 8)) ||
+        (rc = dalloc(&r->d_amax, kModels * 4)) || (rc = dalloc(&r->d_skip, sizeof(T.skip))) || (rc = dalloc(&r->d_stats, (5 + kModels) * 8)) ||
         (rc = dalloc(&r->d_list, size_t(r->P) * 4)) || (rc = dalloc(&r->d_count, 16)) ||
         (rc = dalloc(&r->d_status, sizeof(DevStatus))))
         return fail(rc);
@@ -274,6 +277,8 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
     up(r->d_enc_slot, T.enc_slot, sizeof(T.enc_slot));
     up(r->d_cost, T.cost, sizeof(T.cost));
     up(r->d_amax, amax, sizeof(amax));
+    up(r->d_skip, T.skip, sizeof(T.skip));
+    r->skip_models = T.skip_models;
     if (e == cudaSuccess)
         e = cudaMemsetAsync(r->d_stats, 0, (5 + kModels) * 8, st);
     if (e == cudaSuccess)
@@ -417,20 +422,22 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         return rc;
     rc = timed(r, QEM_K_DECODE_REDUCE, st, [&] {
         return launch_decode_reduce(r->view(), r->tables(), r->d_list, r->d_count, k, rows, d_out, bits / 8,
-                                    r->d_status, r->n_sm, st);
+                                    r->d_status, r->n_sm, st, mode == 1);
     });
     if (rc)
         return rc;
     rc = timed(r, QEM_K_FINALIZE, st, [&] { return launch_copy(bl.d_img, d_out, out_bytes, st); });
     if (rc)
         return rc;
-    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
     bl.state = kValid;
     bl.out_bits = bits;
     bl.pending = true;
     if (used)
         *used = bits;
     if (wait) {
+        // queued (wait == 0) queries leave the status on the device; it accumulates
+        // until qem_finish copies it back
+        QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
         rc = bounded_wait(st);
         if (rc)
             return rc;
@@ -565,8 +572,8 @@ int qem_decode_blocks(qem_resident *r, int64_t first, int64_t n, void *d_out, in
     });
     if (rc)
         return rc;
-    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
     if (wait) {
+        QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
         rc = bounded_wait(st);
         if (rc)
             return rc;

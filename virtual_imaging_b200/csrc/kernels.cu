@@ -38,47 +38,53 @@ __device__ __forceinline__ void report(DevStatus *st, uint32_t flag, long long b
 }
 
 // Forward LSB-first bit reader over aligned 32-bit little-endian words: a
-// 64-bit reservoir `res` holding `n` valid bits.  Loads never pass `last`
-// (the aligned word holding the stream's final byte, plus one), so a
-// malformed stream reads repeated bytes inside its arena instead of running
-// off the end; the caller's length checks then reject it.
+// 64-bit reservoir (lo, hi) holding `n` valid bits.  Words are addressed by
+// index from `first` (the aligned word holding the stream's first byte), and
+// loads never pass word `li` (the aligned word at or after the stream's end),
+// so a malformed stream reads repeated bytes inside its arena instead of
+// running off the end; the caller's length checks then reject it.
 struct Bits {
-    const uint32_t *wp;
-    const uint32_t *last;
     const uint32_t *first;
-    uint64_t res;
+    uint32_t wi;     // next word to load
+    uint32_t li;     // last word that may be loaded
+    uint32_t lo, hi;
     int n;
-    int lead;      // bits of the first word before the stream start
+    int lead;        // bits of the first word before the stream start
 
     __device__ __forceinline__ void init(const uint8_t *p, const uint8_t *end)
     {
         const uintptr_t a = reinterpret_cast<uintptr_t>(p);
-        first = reinterpret_cast<const uint32_t *>(a & ~static_cast<uintptr_t>(3));
-        last = reinterpret_cast<const uint32_t *>((reinterpret_cast<uintptr_t>(end) + 3) &
-                                                  ~static_cast<uintptr_t>(3));
+        const uintptr_t f = a & ~static_cast<uintptr_t>(3);
+        first = reinterpret_cast<const uint32_t *>(f);
+        li = static_cast<uint32_t>((((reinterpret_cast<uintptr_t>(end) + 3) & ~static_cast<uintptr_t>(3)) - f) >> 2);
         lead = static_cast<int>(a & 3) * 8;
-        res = __ldg(first) >> lead;
+        lo = __ldg(first) >> lead;
+        hi = 0u;
         n = 32 - lead;
-        wp = first + 1;
+        wi = 1u;
     }
+    // requires n < 32
     __device__ __forceinline__ void refill()
     {
-        const uint32_t *q = wp < last ? wp : last;
-        res |= static_cast<uint64_t>(__ldg(q)) << n;
+        const uint32_t w = __ldg(first + min(wi, li));
+        lo |= w << n;
+        hi |= n ? (w >> (32 - n)) : 0u;
         n += 32;
-        ++wp;
+        ++wi;
     }
+    // nb < 32 and nb <= n
     __device__ __forceinline__ uint32_t get(int nb)
     {
-        const uint32_t v = static_cast<uint32_t>(res) & ((1u << nb) - 1u);
-        res >>= nb;
+        const uint32_t v = lo & ((1u << nb) - 1u);
+        lo = __funnelshift_r(lo, hi, nb);
+        hi >>= nb;
         n -= nb;
         return v;
     }
     // bits consumed since init
     __device__ __forceinline__ long long consumed() const
     {
-        return 32ll * (wp - first) - lead - n;
+        return 32ll * wi - lead - n;
     }
 };
 
@@ -251,8 +257,35 @@ __device__ __forceinline__ uint32_t tans_step(Stream &S, const uint32_t *dec)
 {
     const uint32_t ent = dec[S.x];
     const int nb = static_cast<int>((ent >> 10) & 15u);
-    S.x = (ent & 1023u) + S.bt.get(nb);
+    S.x = (ent & 1023u) | S.bt.get(nb);      // newbase's low nb bits are zero
     return ent;
+}
+
+// The u8 fast path (paired, no base, no raw bits): one tANS step written out
+// so that the state update, the bit consumption and the packed pair
+// (hi_a | hi_b << 16) cost as few integer-pipe instructions as possible: the
+// table address is formed by mad (FMA pipe), the mask by bmsk, the new state
+// by one lop3 (newbase | (bits & mask); newbase's low nb bits are zero), the
+// reservoir shift by a funnel shift, the pair by prmt.
+__device__ __forceinline__ uint32_t fast_step(uint32_t &x, uint32_t &lo, uint32_t &hi, int &n, uint32_t dec_sa)
+{
+    uint32_t pk, nb;
+    asm("{\n\t"
+        ".reg .b32 a, e, m, t;\n\t"
+        "mad.lo.u32 a, %3, 4, %6;\n\t"
+        "ld.shared.u32 e, [a];\n\t"
+        "bfe.u32 %1, e, 10, 4;\n\t"
+        "bmsk.clamp.b32 m, 0, %1;\n\t"
+        "and.b32 t, %4, m;\n\t"
+        "lop3.b32 %3, e, 1023, t, 0xEA;\n\t"
+        "shf.r.clamp.b32 %4, %4, %5, %1;\n\t"
+        "shr.b32 %5, %5, %1;\n\t"
+        "prmt.b32 %0, e, 0, 0x4342;\n\t"
+        "}"
+        : "=r"(pk), "=r"(nb), "+r"(n), "+r"(x), "+r"(lo), "+r"(hi)
+        : "r"(dec_sa));
+    n -= static_cast<int>(nb);
+    return pk;
 }
 
 // Decode 16 pairs (32 scans) of a paired stream into values v[32] (general
@@ -652,48 +685,56 @@ __global__ void __launch_bounds__(256) k_enc_compact(const T *__restrict__ count
 // ---------------------------------------------------------------------------
 // a5: plan
 // ---------------------------------------------------------------------------
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;
 
+// Blocks [0, n_list_blocks) build the pixel list, one pixel per thread: a
+// warp ballots its 32 pixels and reserves room in the list with one atomic
+// on *count (zeroed by the host before the launch).  The list is in ascending
+// order within each warp's run; runs land in any order, which the sums do not
+// see (integer addition).  Full query: mask && valid; delta: pixels whose
+// (mask && valid) changed against the stored baseline mask, leaving pixels
+// flagged in bit 31.  Every thread then stores the new mask as the baseline.
+// Blocks past n_list_blocks initialise the output rows (0, or the baseline
+// image for a delta).
 __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict__ mask,
                                                       const uint8_t *__restrict__ valid,
                                                       uint8_t *__restrict__ base_mask, int P, int mode,
-                                                      uint32_t *__restrict__ list, uint32_t *__restrict__ count,
-                                                      uint4 *__restrict__ out, const uint4 *__restrict__ base_img,
-                                                      long long n_vec)
+                                                      int n_list_blocks, uint32_t *__restrict__ list,
+                                                      uint32_t *__restrict__ count, uint4 *__restrict__ out,
+                                                      const uint4 *__restrict__ base_img, long long n_vec)
 {
-    if (blockIdx.x == 0) {
-        __shared__ uint32_t s_warp[32];
-        const int per = (P + kPlanThreads - 1) / kPlanThreads;
-        const int p0 = min(P, static_cast<int>(threadIdx.x) * per);
-        const int p1 = min(P, p0 + per);
-        uint32_t local = 0;
-        for (int p = p0; p < p1; ++p) {
+    if (static_cast<int>(blockIdx.x) < n_list_blocks) {
+        const int p = static_cast<int>(blockIdx.x) * kPlanThreads + static_cast<int>(threadIdx.x);
+        const int lane = threadIdx.x & 31;
+        bool emit = false;
+        uint32_t entry = 0;
+        uint8_t mk = 0;
+        if (p < P) {
             const bool ok = valid[p] != 0;
-            const bool nw = ok && mask[p] != 0;
-            const bool od = ok && base_mask[p] != 0;
-            local += mode == 0 ? nw : (nw != od);
-        }
-        uint32_t total;
-        uint32_t pos = block_exclusive_scan(local, s_warp, total);
-        for (int p = p0; p < p1; ++p) {
-            const bool ok = valid[p] != 0;
-            const uint8_t mk = mask[p];
+            mk = mask[p];
             const bool nw = ok && mk != 0;
             const bool od = ok && base_mask[p] != 0;
             if (mode == 0) {
-                if (nw)
-                    list[pos++] = static_cast<uint32_t>(p);
-            } else if (nw != od) {
-                list[pos++] = static_cast<uint32_t>(p) | (od ? 0x80000000u : 0u);
+                emit = nw;
+                entry = static_cast<uint32_t>(p);
+            } else {
+                emit = nw != od;
+                entry = static_cast<uint32_t>(p) | (od ? 0x80000000u : 0u);
             }
             base_mask[p] = mk;
         }
-        if (threadIdx.x == 0)
-            *count = total;
+        const unsigned bal = __ballot_sync(kFull, emit);
+        uint32_t at = 0;
+        if (lane == 0 && bal)
+            at = atomicAdd(count, static_cast<uint32_t>(__popc(bal)));
+        at = __shfl_sync(kFull, at, 0);
+        if (emit)
+            list[at + __popc(bal & ((1u << lane) - 1u))] = entry;
         return;
     }
-    const long long stride = static_cast<long long>(gridDim.x - 1) * blockDim.x;
-    for (long long i = static_cast<long long>(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n_vec; i += stride)
+    const long long stride = static_cast<long long>(gridDim.x - n_list_blocks) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x - n_list_blocks) * blockDim.x + threadIdx.x; i < n_vec;
+         i += stride)
         out[i] = mode == 0 ? make_uint4(0u, 0u, 0u, 0u) : base_img[i];
 }
 
@@ -714,16 +755,17 @@ __global__ void k_copy(uint4 *__restrict__ dst, const uint4 *__restrict__ src, l
 // across the warp with redux.sync, adding each scan's total into a per-row
 // shared accumulator; the CTA then adds its rows to the output with one
 // global atomic per nonzero scan sum.
-template <int W>
-__device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint32_t *list,
-                                            uint32_t n, int tile, long long b, uint32_t *acc, int lane,
-                                            DevStatus *st)
+template <int W, bool DELTA>
+__device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint16_t *skip,
+                                            uint32_t skip_models, const uint32_t *list, uint32_t n, int tile,
+                                            long long b, uint32_t *acc, uint32_t *stage, uint32_t *cnt,
+                                            int lane, DevStatus *st)
 {
     const uint32_t idx = static_cast<uint32_t>(tile) * 32u + static_cast<uint32_t>(lane);
     const bool listed = idx < n;
     const uint32_t e = listed ? __ldg(list + idx) : 0u;
     const int p = static_cast<int>(e & 0x7FFFFFFFu);
-    const bool neg = (e >> 31) != 0u;
+    const bool neg = DELTA && (e >> 31) != 0u;
     Stream S;
     S.form = kEmpty;
     S.model = 0;
@@ -743,32 +785,40 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     const unsigned nact = __popc(__ballot_sync(kFull, listed));
     if (lane == 0) {
         if (tile == 0)
-            atomicAdd(&st->rows, 1ull);
-        atomicAdd(&st->streams, static_cast<unsigned long long>(nact));
+            atomicAdd(cnt, 1u);
+        atomicAdd(cnt + 1, nact);
     }
 
     const uint32_t *dec = s_dec + S.model * kStates;
-    const bool fast = S.form == kPaired && S.shift == 0 && S.base == 0u;
+    // low-dose paired streams (models dominated by the (0,0) symbol) are decoded
+    // by runs after the per-scan loop instead of inside it
+    const bool runs = S.form == kPaired && S.shift == 0 && S.base == 0u && ((skip_models >> S.model) & 1u);
+    const bool dense_lane = (S.form == kPaired && !runs) || S.form == kLiteral || S.form == kConstant;
+    const bool fast = S.form == kPaired && !runs && S.shift == 0 && S.base == 0u;
     uint32_t over = 0;
+    // warps whose lanes hold only empty, sparse or run-decoded streams skip the per-scan loop
+    const bool dense = __any_sync(kFull, dense_lane);
 
     if (W == 1) {
         // counts fit 16-bit halves: pack scans (2j, 2j+1) into one word; a
         // leaving pixel contributes 255 - v per half and the warp subtracts
         // 255 x (number of such lanes) afterwards.
-        const bool packed_src = S.form == kPaired || S.form == kLiteral || S.form == kConstant;
+        const bool packed_src = dense_lane;
         const uint32_t flip = (neg && packed_src) ? 0x00FF00FFu : 0u;
         const uint32_t corr = 255u * static_cast<uint32_t>(__popc(__ballot_sync(kFull, neg && packed_src)));
         const uint32_t cpk = S.form == kConstant ? (S.c | (S.c << 16)) : 0u;
-        for (int seg = 0; seg < 16; ++seg) {
+        const uint32_t dec_sa = static_cast<uint32_t>(__cvta_generic_to_shared(dec));
+        for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
             uint32_t pk[16];
             if (fast) {
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
+                    // top-ups before steps 0, 3, 6, 9, 12, 15: <= 30 bits per 3 steps
                     if (jj % 3 == 0 && S.bt.n < 30)
                         S.bt.refill();
-                    pk[jj] = __byte_perm(tans_step(S, dec), 0u, 0x4342);
+                    pk[jj] = fast_step(S.x, S.bt.lo, S.bt.hi, S.bt.n, dec_sa);
                 }
-            } else if (S.form == kPaired) {
+            } else if (S.form == kPaired && !runs) {
                 uint32_t vv[32];
                 paired_segment(S, dec, vv, over);
 #pragma unroll
@@ -788,22 +838,26 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                 for (int jj = 0; jj < 16; ++jj)
                     pk[jj] = cpk;
             }
-            uint32_t mine = 0;
+            // warp sums of the 16 packed pairs are warp-uniform: one lane
+            // parks them in shared memory, every lane then takes its scan
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
-                const uint32_t r = __reduce_add_sync(kFull, pk[jj] ^ flip);
-                if ((lane >> 1) == jj)
-                    mine = r;
+                const uint32_t r = __reduce_add_sync(kFull, DELTA ? (pk[jj] ^ flip) : pk[jj]);
+                if (lane == 0)
+                    stage[jj] = r;
             }
-            mine = ((lane & 1) ? (mine >> 16) : (mine & 0xFFFFu)) - corr;
+            __syncwarp();
+            uint32_t mine = stage[lane >> 1];
+            __syncwarp();
+            mine = ((lane & 1) ? (mine >> 16) : (mine & 0xFFFFu)) - (DELTA ? corr : 0u);
             if (mine)
                 atomicAdd(acc + seg * 32 + lane, mine);
         }
     } else {
         const uint32_t sgn = neg ? 0xFFFFFFFFu : 0u;       // v -> (v ^ sgn) - sgn negates
-        for (int seg = 0; seg < 16; ++seg) {
+        for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
             uint32_t vv[32];
-            if (S.form == kPaired) {
+            if (S.form == kPaired && !runs) {
                 paired_segment(S, dec, vv, over);
             } else if (S.form == kLiteral) {
 #pragma unroll
@@ -821,7 +875,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
             uint32_t mine = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const uint32_t r = __reduce_add_sync(kFull, (vv[i] ^ sgn) - sgn);
+                const uint32_t r = __reduce_add_sync(kFull, DELTA ? (vv[i] ^ sgn) - sgn : vv[i]);
                 if (lane == i)
                     mine = r;
             }
@@ -830,7 +884,45 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
         }
     }
 
-    if (S.form == kPaired) {
+    if (runs) {
+        // Runs of zero-bit (0,0) steps are jumped with one table read; every
+        // other step is an ordinary tANS step whose nonzero counts are added
+        // to their scans.  A run that would pass pair 255 cannot end in the
+        // final state 1024 (that state reads bits), so it marks the stream
+        // malformed.  Each iteration advances j, so the loop ends.
+        const uint16_t *sk = skip + S.model * kStates;
+        int j = 0;
+        bool bad = false;
+        while (j < kPairs) {
+            // a maximal run ends on a slot that reads bits or carries another
+            // symbol, so every iteration is: jump the run (if any), then one step
+            const uint32_t r = sk[S.x];
+            const int run = static_cast<int>(r >> 10);
+            if (run) {
+                j += run;
+                S.x = r & 1023u;
+                if (j >= kPairs) {
+                    bad = j > kPairs;
+                    break;
+                }
+                if (run == 63)
+                    continue;      // a capped run may go on from the slot it reached
+            }
+            if (S.bt.n < 10)
+                S.bt.refill();
+            const uint32_t ent = tans_step(S, dec);
+            const uint32_t a = (ent >> 16) & 0xFFu, c = ent >> 24;
+            if (a)
+                atomicAdd(acc + 2 * j, neg ? 0u - a : a);
+            if (c)
+                atomicAdd(acc + 2 * j + 1, neg ? 0u - c : c);
+            ++j;
+        }
+        if (bad)
+            report(st, kErrState, b, p);
+        else
+            close_paired(S, b, p, st);
+    } else if (S.form == kPaired) {
         if (over > (W == 1 ? 0xFFu : 0xFFFFu)) {
             report(st, kErrValue, b, p);
         }
@@ -867,23 +959,43 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     }
 }
 
-template <int W, int THREADS>
+constexpr int kMaxSlots = 8;    // block rows one CTA range may touch (shared accumulators)
+
+template <int W, int THREADS, bool DELTA>
 __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint32_t *__restrict__ dec_g,
+                                                             const uint16_t *__restrict__ skip_g,
+                                                             uint32_t skip_models, int skip_count,
                                                              const uint32_t *__restrict__ list,
                                                              const uint32_t *__restrict__ count, int stride,
                                                              long long rows, void *__restrict__ out,
                                                              int out_bytes, DevStatus *__restrict__ st)
 {
-    constexpr int WARPS = THREADS / 32;
+    constexpr int MAXW = THREADS / 32;
+    // shared memory: decode tables of the 32 models | run tables of the first
+    // skip_count models | kMaxSlots per-row scan accumulators
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *s_dec = smem;
-    uint32_t *s_acc = smem + kModels * kStates;
+    uint16_t *s_skip = reinterpret_cast<uint16_t *>(smem + kModels * kStates);
+    uint32_t *s_stage = smem + kModels * kStates + skip_count * kStates / 2;   // 16 words per warp
+    uint32_t *s_acc = s_stage + MAXW * 16;
     for (int i = threadIdx.x; i < kModels * kStates / 4; i += THREADS)
         reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
+    for (int i = threadIdx.x; i < skip_count * kStates / 8; i += THREADS)
+        reinterpret_cast<uint4 *>(s_skip)[i] = __ldg(reinterpret_cast<const uint4 *>(skip_g) + i);
+    // per-CTA counters (rows, streams), added to the status once at the end
+    __shared__ uint32_t s_cnt[2];
+    if (threadIdx.x < 2)
+        s_cnt[threadIdx.x] = 0u;
 
     const uint32_t n = __ldg(count);
     const long long tiles = (n + 31u) >> 5;
     const long long total = rows * tiles;
+    // tasks per CTA range: up to one per warp, fewer when that spreads the work
+    // over more SMs, and few enough that a range touches at most kMaxSlots rows
+    const long long per = (total + gridDim.x - 1) / gridDim.x;
+    long long cap = (kMaxSlots - 1) * tiles + 1;
+    cap = cap < MAXW ? cap : MAXW;
+    const int WARPS = static_cast<int>(per < 1 ? 1 : (per > cap ? cap : per));
     const long long ranges = (total + WARPS - 1) / WARPS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (long long r = blockIdx.x; r < ranges; r += gridDim.x) {
@@ -895,10 +1007,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
             s_acc[i] = 0u;
         __syncthreads();
         const long long task = t0 + warp;
-        if (task < total) {
+        if (warp < WARPS && task < total) {
             const long long row = task / tiles;
             const int tile = static_cast<int>(task - row * tiles);
-            decode_task<W>(v, s_dec, list, n, tile, row * stride, s_acc + (row - row0) * kScans, lane, st);
+            decode_task<W, DELTA>(v, s_dec, s_skip, skip_models, list, n, tile, row * stride,
+                                  s_acc + (row - row0) * kScans, s_stage + warp * 16, s_cnt, lane, st);
         }
         __syncthreads();
         for (int i = threadIdx.x; i < nslot * kScans; i += THREADS) {
@@ -913,6 +1026,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
             }
         }
         __syncthreads();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && (s_cnt[0] | s_cnt[1])) {
+        atomicAdd(&st->rows, static_cast<unsigned long long>(s_cnt[0]));
+        atomicAdd(&st->streams, static_cast<unsigned long long>(s_cnt[1]));
     }
 }
 
@@ -1090,11 +1208,15 @@ cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, uint8_t *base
                         int out_bytes, cudaStream_t st)
 {
     const long long n_vec = n_elems * out_bytes / 16;
-    int fill = static_cast<int>((n_vec + kPlanThreads - 1) / kPlanThreads);
-    fill = fill < 1 ? 1 : (fill > 4 * sm_count() ? 4 * sm_count() : fill);
-    k_plan<<<1 + fill, kPlanThreads, 0, st>>>(mask, valid, base_mask, P, mode, list, count,
-                                              static_cast<uint4 *>(out), static_cast<const uint4 *>(base_img),
-                                              n_vec);
+    const int n_list = (P + kPlanThreads - 1) / kPlanThreads;
+    int fill = static_cast<int>((n_vec + kPlanThreads * 4 - 1) / (kPlanThreads * 4));
+    fill = fill < 1 ? 1 : (fill > 8 * sm_count() ? 8 * sm_count() : fill);
+    cudaError_t e = cudaMemsetAsync(count, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess)
+        return e;
+    k_plan<<<n_list + fill, kPlanThreads, 0, st>>>(mask, valid, base_mask, P, mode, n_list, list, count,
+                                                   static_cast<uint4 *>(out), static_cast<const uint4 *>(base_img),
+                                                   n_vec);
     return cudaGetLastError();
 }
 
@@ -1107,34 +1229,37 @@ cudaError_t launch_copy(void *dst, const void *src, size_t bytes, cudaStream_t s
     return cudaGetLastError();
 }
 
+template <int W, int TH, bool DELTA>
+cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride, long long rows,
+                      void *out, int out_bytes, DevStatus *status, int n_sm, cudaStream_t st)
+{
+    // the run-decoded models are a prefix 0..k-1 (their (0,0) share falls as lambda grows)
+    const int skip_count = __builtin_popcount(tb.skip_models);
+    const size_t smem = kTableBytes + static_cast<size_t>(skip_count) * kStates * sizeof(uint16_t) +
+                        static_cast<size_t>(TH / 32) * 16 * sizeof(uint32_t) +
+                        static_cast<size_t>(kMaxSlots) * kScans * sizeof(uint32_t);
+    static size_t attr = 0;
+    if (attr < smem) {
+        const cudaError_t e = cudaFuncSetAttribute(k_decode_reduce<W, TH, DELTA>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess)
+            return e;
+        attr = smem;
+    }
+    k_decode_reduce<W, TH, DELTA><<<n_sm, TH, smem, st>>>(v, tb.dec, tb.skip, tb.skip_models, skip_count, list,
+                                                          count, stride, rows, out, out_bytes, status);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride,
                                  long long rows, void *out, int out_bytes, DevStatus *status, int n_sm,
-                                 cudaStream_t st)
+                                 cudaStream_t st, bool delta)
 {
-    if (v.w == 1) {
-        constexpr int TH = 1024;
-        const size_t smem = kTableBytes + static_cast<size_t>(TH / 32) * kScans * sizeof(uint32_t);
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(k_decode_reduce<1, TH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-            attr = true;
-        }
-        k_decode_reduce<1, TH><<<n_sm, TH, smem, st>>>(v, tb.dec, list, count, stride, rows, out, out_bytes,
-                                                       status);
-    } else {
-        constexpr int TH = 512;
-        const size_t smem = kTableBytes + static_cast<size_t>(TH / 32) * kScans * sizeof(uint32_t);
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(k_decode_reduce<2, TH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-            attr = true;
-        }
-        k_decode_reduce<2, TH><<<n_sm, TH, smem, st>>>(v, tb.dec, list, count, stride, rows, out, out_bytes,
-                                                       status);
-    }
-    return cudaGetLastError();
+    if (v.w == 1)
+        return delta ? launch_dr<1, 1024, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
+                     : launch_dr<1, 1024, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
+    return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
+                 : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
 }
 
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,

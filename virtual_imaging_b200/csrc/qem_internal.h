@@ -56,6 +56,8 @@ struct Tables {
     const uint16_t *enc_slot;
     const uint32_t *cost;
     const uint32_t *amax;
+    const uint16_t *skip;     // [m][slot]: run of zero-bit (0,0) steps from slot (bits 10-15, <= 63), slot after it (bits 0-9)
+    uint32_t skip_models;     // bit m set: model m's streams are decoded by runs
 };
 
 struct HostTables {
@@ -65,6 +67,8 @@ struct HostTables {
     uint32_t dec[kModels][kStates];
     uint32_t enc_sym[kModels][256];
     uint16_t enc_slot[kModels][kStates];
+    uint16_t skip[kModels][kStates];
+    uint32_t skip_models;
 };
 
 // What the query kernels read of a resident.
@@ -117,7 +121,7 @@ cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, uint8_t *base
                         cudaStream_t st);
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count,
                                  int stride, long long rows, void *out, int out_bytes,
-                                 DevStatus *status, int n_sm, cudaStream_t st);
+                                 DevStatus *status, int n_sm, cudaStream_t st, bool delta = false);
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, cudaStream_t st);
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out,
                                  DevStatus *status, cudaStream_t st);

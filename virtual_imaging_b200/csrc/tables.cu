@@ -126,6 +126,39 @@ void make_model(int m, HostTables &T)
     }
 }
 
+// Runs of zero-bit (0,0) steps.  A slot whose symbol is (0,0) and whose
+// entry reads no bits moves the decoder, deterministically, to slot newbase,
+// which is strictly lower (newbase = f + rank - 1024 <= slot - (1024 - f)),
+// so the runs follow from one ascending pass.  skip[slot] (16 bits): the run
+// length from this slot, capped at 63, in bits 10-15, and the slot reached
+// after that many steps in bits 0-9; 0 when the slot itself reads bits or
+// carries another symbol.  A capped run continues from the slot it reaches.
+void make_runs(int m, HostTables &T)
+{
+    std::array<int, kStates> run{}, next{};
+    for (int slot = 0; slot < kStates; ++slot) {
+        const uint32_t e = T.dec[m][slot];
+        const uint32_t nb = (e >> 10) & 15u, sym = e >> 16, nx = e & 1023u;
+        next[slot] = -1;
+        if (sym == 0u && nb == 0u && nx < static_cast<uint32_t>(slot)) {
+            next[slot] = static_cast<int>(nx);
+            run[slot] = 1 + run[nx];
+        }
+    }
+    for (int slot = 0; slot < kStates; ++slot) {
+        const int r = run[slot] < 63 ? run[slot] : 63;
+        int at = slot;
+        for (int k = 0; k < r; ++k)
+            at = next[at];
+        T.skip[m][slot] = r ? static_cast<uint16_t>((r << 10) | at) : static_cast<uint16_t>(0);
+    }
+    // decode by runs only where (0,0) holds at least 7/8 of the states (lambda
+    // up to ~0.04 here), a prefix of at most 8 models whose run tables live in
+    // shared memory; there a stream needs ~30-100 events instead of 256 steps
+    if (T.freq[m][0] >= 896 && m < 8 && (m == 0 || ((T.skip_models >> (m - 1)) & 1u)))
+        T.skip_models |= 1u << m;
+}
+
 }  // namespace
 
 const HostTables &host_tables()
@@ -135,6 +168,9 @@ const HostTables &host_tables()
     std::call_once(once, [] {
         for (int m = 0; m < kModels; ++m)
             make_model(m, tables);
+        tables.skip_models = 0u;
+        for (int m = 0; m < kModels; ++m)
+            make_runs(m, tables);
     });
     return tables;
 }
