@@ -267,6 +267,10 @@ def run_profile_case(dev, torch, V):
     res.profile(True)
     for m in (bf, adf, bf, adf):
         res.masked_sum(m, out=out)
+    # a short drag: one full query then delta queries (launches 5.. are deltas)
+    for t, d in enumerate(w.drag[:6]):
+        md = torch.from_numpy(d).to(dev)
+        (res.masked_sum_delta if t else res.masked_sum)(md, out=out)
     p = res.profile_read()
     print(json.dumps({"encode_s": t_enc, "kernels": p}), flush=True)
     res.free()

@@ -123,17 +123,17 @@ def _check(code: int, where: str):
     raise QemError(code, where)
 
 
-def _stream(stream=None) -> ctypes.c_void_p:
+def _stream(stream=None) -> int:
     s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    return s.cuda_stream
 
 
-def _dev_ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+def _dev_ptr(t: torch.Tensor | None) -> int:
     if t is None:
-        return ctypes.c_void_p(0)
+        return 0
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError("expected a contiguous CUDA tensor")
-    return ctypes.c_void_p(t.data_ptr())
+    return t.data_ptr()
 
 
 def _count_dtype(bits: int):
@@ -156,6 +156,14 @@ class Resident:
 
     def __init__(self, handle: ctypes.c_void_p):
         self._h = handle
+        self._geom = None
+
+    def _static(self):
+        """(n_blocks, n_pixels, dtype_bits, out_bits_auto): fixed once the resident exists."""
+        if self._geom is None:
+            i = self.info()
+            self._geom = (i["n_blocks"], i["n_pixels"], i["dtype_bits"], i["out_bits_auto"])
+        return self._geom
 
     # ---- construction -------------------------------------------------------
     @classmethod
@@ -200,13 +208,12 @@ class Resident:
 
     # ---- queries ---------------------------------------------------------------
     def _query(self, fn, name, mask, block_stride, out_bits, out, wait, stream):
-        info = self.info()
-        rows = -(-info["n_blocks"] // block_stride)
-        bits = info["out_bits_auto"] if out_bits == 0 else out_bits
         if out is None:
+            n_blocks, _, _, auto = self._static()
+            rows = -(-n_blocks // block_stride)
+            bits = auto if out_bits == 0 else out_bits
             out = torch.empty((rows, 512), dtype=out_dtype(bits), device=mask.device)
-        used = ctypes.c_int32(0)
-        _check(fn(self._h, _dev_ptr(mask), block_stride, out_bits, _dev_ptr(out), ctypes.byref(used),
+        _check(fn(self._h, _dev_ptr(mask), block_stride, out_bits, _dev_ptr(out), None,
                   1 if wait else 0, _stream(stream)), name)
         return out
 
@@ -232,9 +239,9 @@ class Resident:
 
     def decode_blocks(self, first: int, n: int, out: torch.Tensor | None = None, wait: bool = True,
                       stream=None) -> torch.Tensor:
-        info = self.info()
         if out is None:
-            out = torch.empty((n * 512, info["n_pixels"]), dtype=_count_dtype(info["dtype_bits"]),
+            _, n_pixels, bits, _ = self._static()
+            out = torch.empty((n * 512, n_pixels), dtype=_count_dtype(bits),
                               device=torch.device("cuda", torch.cuda.current_device()))
         _check(lib().qem_decode_blocks(self._h, first, n, _dev_ptr(out), 1 if wait else 0, _stream(stream)),
                "qem_decode_blocks")

@@ -133,6 +133,18 @@ __device__ __forceinline__ bool locate(const View &v, long long b, int p, const 
     return true;
 }
 
+// Ask L2 for every 128-byte line of a stream up front: the decoder then
+// reads it word by word along a dependent chain, and each of those reads
+// would otherwise wait for HBM.  Prefetches take no registers and never fault.
+__device__ __forceinline__ void prefetch_stream(const uint8_t *s, uint32_t len)
+{
+    // lines after the one holding the header (that one is being read already)
+    const uintptr_t a = (reinterpret_cast<uintptr_t>(s) & ~static_cast<uintptr_t>(127)) + 128;
+    const uintptr_t e = reinterpret_cast<uintptr_t>(s) + len;
+    for (uintptr_t q = a; q < e; q += 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(q));
+}
+
 // Parse the header and set the readers up; false (after reporting) if malformed.
 __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
 {
@@ -140,6 +152,7 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
         S.form = kEmpty;
         return true;
     }
+    prefetch_stream(S.s, S.len);
     if (S.len < 2) {
         report(st, kErrLength, b, p);
         return false;
