@@ -299,6 +299,7 @@ def main():
     import torch.distributed as dist
 
     import virtual_imaging_b200 as V
+    from virtual_imaging_b200.series import max_over_ranks
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -372,10 +373,7 @@ def main():
     t = e0.elapsed_time(e1) / 1e3
     prof = res.profile_read()
     res.profile(False)
-    if world > 1:
-        tt = torch.tensor([t], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
+    t = max_over_ranks(t, device=dev)
 
     # end to end: masks from pinned host memory in, images to pinned host memory out
     host_masks = [torch.from_numpy(m.astype(np.uint8)).pin_memory() for (_, m, _, _) in sched]
@@ -404,10 +402,7 @@ def main():
     torch.cuda.synchronize()
     res.finish()
     te = f0.elapsed_time(f1) / 1e3
-    if world > 1:
-        tt = torch.tensor([te], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        te = float(tt.item())
+    te = max_over_ranks(te, device=dev)
 
     # per-query breakdown (separate, untimed for `value`)
     lens = stream_lengths(res, w)
