@@ -55,6 +55,7 @@ struct qem_resident {
     int n_sm = 1;
 
     uint8_t *d_valid = nullptr;
+    uint8_t *d_pclass = nullptr;                // per pixel: 1 = light streams (from block 0)
     uint32_t *d_groups = nullptr;
     unsigned long long *d_blk_ptr = nullptr;
     uint32_t *d_blk_len = nullptr;
@@ -176,6 +177,7 @@ void release(qem_resident *r)
         cudaFree(kv.second.d_img);
     }
     cudaFree(r->d_valid);
+    cudaFree(r->d_pclass);
     cudaFree(r->d_groups);
     cudaFree(r->d_blk_ptr);
     cudaFree(r->d_blk_len);
@@ -252,7 +254,7 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
     r->out_bits_auto = static_cast<uint64_t>(r->n_valid) * ((1ull << bits) - 1ull) > 0xFFFFFFFFull ? 64 : 32;
 
     const HostTables &T = host_tables();
-    if ((rc = dalloc(&r->d_valid, hv.size())) || (rc = dalloc(&r->d_groups, size_t(r->B) * r->G * kGroupWords * 4)) ||
+    if ((rc = dalloc(&r->d_valid, hv.size())) || (rc = dalloc(&r->d_pclass, hv.size())) || (rc = dalloc(&r->d_groups, size_t(r->B) * r->G * kGroupWords * 4)) ||
         (rc = dalloc(&r->d_blk_ptr, size_t(r->B) * 8)) || (rc = dalloc(&r->d_blk_len, size_t(r->B) * 4)) ||
         (rc = dalloc(&r->d_dec, sizeof(T.dec))) || (rc = dalloc(&r->d_enc_sym, sizeof(T.enc_sym))) ||
         (rc = dalloc(&r->d_enc_slot, sizeof(T.enc_slot))) || (rc = dalloc(&r->d_cost, sizeof(T.cost))) ||
@@ -279,6 +281,8 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
     up(r->d_amax, amax, sizeof(amax));
     up(r->d_skip, T.skip, sizeof(T.skip));
     r->skip_models = T.skip_models;
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(r->d_pclass, 0, hv.size(), st);
     if (e == cudaSuccess)
         e = cudaMemsetAsync(r->d_stats, 0, (5 + kModels) * 8, st);
     if (e == cudaSuccess)
@@ -415,8 +419,8 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
             mode = 1;
     }
     int rc = timed(r, QEM_K_PLAN, st, [&] {
-        return launch_plan(d_mask, r->d_valid, bl.d_mask, r->P, mode, r->d_list, r->d_count, d_out, bl.d_img,
-                           n_elems, bits / 8, st);
+        return launch_plan(d_mask, r->d_valid, r->d_pclass, bl.d_mask, r->P, mode, r->d_list, r->d_count, d_out,
+                           bl.d_img, n_elems, bits / 8, st);
     });
     if (rc)
         return rc;
@@ -497,7 +501,8 @@ int qem_encode_append(qem_resident *r, const void *d_counts, int64_t n_blocks, v
         const void *counts = src + static_cast<size_t>(done) * block_raw;
         const int64_t b0 = r->B_done;
         rc = timed(r, QEM_K_ENC_STREAMS, st, [&] {
-            return launch_enc_streams(counts, r->w, r->P, nb, r->tables(), r->d_desc, r->d_slots, r->d_stats, st);
+            return launch_enc_streams(counts, r->w, r->P, nb, r->tables(), r->d_desc, r->d_slots, r->d_stats,
+                                      b0 == 0 ? r->d_pclass : nullptr, st);
         });
         if (rc)
             return rc;
@@ -734,6 +739,7 @@ int qem_import(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t d
     if (e == cudaSuccess && total)
         e = cudaMemcpy(a.p, h_payload + h_block_off[0], total, cudaMemcpyHostToDevice);
     std::vector<uint32_t> lens(static_cast<size_t>(r->B));
+    std::vector<uint8_t> pclass0(static_cast<size_t>(r->P), 1);   // empty streams are light
     for (int64_t b = 0; b < r->B; ++b) {
         r->blk_ptr[b] = reinterpret_cast<unsigned long long>(a.p + (h_block_off[b] - h_block_off[0]));
         r->blk_len[b] = h_block_off[b + 1] - h_block_off[b];
@@ -752,6 +758,12 @@ int qem_import(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t d
                 continue;
             }
             const int form = pl[st0] & 7;
+            if (b == 0) {
+                const uint32_t hdr = pl[st0] | (uint32_t(pl[st0 + 1]) << 8);
+                const bool runs = form == kPaired && ((hdr >> 8) & 0x1Fu) == 0u &&
+                                  ((r->skip_models >> ((hdr >> 3) & 31u)) & 1u);
+                pclass0[px] = (form == kSparse || runs) ? 1 : 0;
+            }
             if (form >= 1 && form <= 4) {
                 r->form_count[form] += 1;
                 if (form == kPaired)
@@ -765,6 +777,8 @@ int qem_import(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t d
         e = cudaMemcpy(r->d_blk_ptr, r->blk_ptr.data(), size_t(r->B) * 8, cudaMemcpyHostToDevice);
     if (e == cudaSuccess)
         e = cudaMemcpy(r->d_blk_len, lens.data(), size_t(r->B) * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(r->d_pclass, pclass0.data(), pclass0.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess)
         return fail(cuda_status(e));
     r->B_done = r->B;

@@ -379,7 +379,8 @@ template <typename T>
 __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict__ counts, int P, int nblk,
                                                             Tables tb, uint4 *__restrict__ desc,
                                                             uint32_t *__restrict__ slots,
-                                                            unsigned long long *__restrict__ stats)
+                                                            unsigned long long *__restrict__ stats,
+                                                            uint8_t *__restrict__ pclass)
 {
     constexpr uint32_t W = sizeof(T);
     __shared__ uint32_t s_cost[kModels * 16];
@@ -518,6 +519,14 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
             d.z = base | (nnz << 16);
         }
         desc[sid] = d;
+        if (pclass && b == 0) {
+            // the pixel's cost class, from its block-0 stream: 1 = light (empty,
+            // sparse, or paired decoded by runs), 0 = heavy (decoded pair by pair)
+            const uint32_t hdr = d.y & 0xFFFFu;
+            const bool runs = form == kPaired && ((hdr >> 8) & 0x1Fu) == 0u &&
+                              ((tb.skip_models >> model) & 1u);
+            pclass[p] = (form == kEmpty || form == kSparse || runs) ? 1 : 0;
+        }
         atomicAdd(&s_stats[form], 1u);
         if (form == kPaired)
             atomicAdd(&s_stats[5 + model], 1u);
@@ -701,16 +710,18 @@ __global__ void __launch_bounds__(256) k_enc_compact(const T *__restrict__ count
 constexpr int kPlanThreads = 256;
 
 // Blocks [0, n_list_blocks) build the pixel list, one pixel per thread: a
-// warp ballots its 32 pixels and reserves room in the list with one atomic
-// on *count (zeroed by the host before the launch).  The list is in ascending
-// order within each warp's run; runs land in any order, which the sums do not
-// see (integer addition).  Full query: mask && valid; delta: pixels whose
-// (mask && valid) changed against the stored baseline mask, leaving pixels
-// flagged in bit 31.  Every thread then stores the new mask as the baseline.
-// Blocks past n_list_blocks initialise the output rows (0, or the baseline
-// image for a delta).
+// warp ballots its 32 pixels and reserves room with one atomic per class.
+// Pixels of the heavy class (decoded pair by pair) fill the list from the
+// front (count[0]), light ones (empty, sparse, run-decoded) from the back
+// (count[1], list[P-1], list[P-2], ...), so that warps meet one kind of work.
+// Order inside a class does not matter to the sums (integer addition).
+// Full query: mask && valid; delta: pixels whose (mask && valid) changed
+// against the stored baseline mask, leaving pixels flagged in bit 31.  Every
+// thread then stores the new mask as the baseline.  Blocks past n_list_blocks
+// initialise the output rows (0, or the baseline image for a delta).
 __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict__ mask,
                                                       const uint8_t *__restrict__ valid,
+                                                      const uint8_t *__restrict__ pclass,
                                                       uint8_t *__restrict__ base_mask, int P, int mode,
                                                       int n_list_blocks, uint32_t *__restrict__ list,
                                                       uint32_t *__restrict__ count, uint4 *__restrict__ out,
@@ -719,7 +730,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
     if (static_cast<int>(blockIdx.x) < n_list_blocks) {
         const int p = static_cast<int>(blockIdx.x) * kPlanThreads + static_cast<int>(threadIdx.x);
         const int lane = threadIdx.x & 31;
-        bool emit = false;
+        bool emit = false, light = false;
         uint32_t entry = 0;
         uint8_t mk = 0;
         if (p < P) {
@@ -734,15 +745,23 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
                 emit = nw != od;
                 entry = static_cast<uint32_t>(p) | (od ? 0x80000000u : 0u);
             }
+            light = pclass[p] != 0;
             base_mask[p] = mk;
         }
-        const unsigned bal = __ballot_sync(kFull, emit);
+        const unsigned bh = __ballot_sync(kFull, emit && !light);
+        const unsigned bl = __ballot_sync(kFull, emit && light);
         uint32_t at = 0;
-        if (lane == 0 && bal)
-            at = atomicAdd(count, static_cast<uint32_t>(__popc(bal)));
-        at = __shfl_sync(kFull, at, 0);
-        if (emit)
-            list[at + __popc(bal & ((1u << lane) - 1u))] = entry;
+        if (lane == 0 && bh)
+            at = atomicAdd(count, static_cast<uint32_t>(__popc(bh)));
+        if (lane == 1 && bl)
+            at = atomicAdd(count + 1, static_cast<uint32_t>(__popc(bl)));
+        const uint32_t ah = __shfl_sync(kFull, at, 0);
+        const uint32_t al = __shfl_sync(kFull, at, 1);
+        const unsigned below = (1u << lane) - 1u;
+        if (emit && !light)
+            list[ah + __popc(bh & below)] = entry;
+        if (emit && light)
+            list[P - 1 - (al + __popc(bl & below))] = entry;
         return;
     }
     const long long stride = static_cast<long long>(gridDim.x - n_list_blocks) * blockDim.x;
@@ -770,12 +789,25 @@ __global__ void k_copy(uint4 *__restrict__ dst, const uint4 *__restrict__ src, l
 // global atomic per nonzero scan sum.
 template <int W, bool DELTA>
 __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint16_t *skip,
-                                            uint32_t skip_models, const uint32_t *list, uint32_t n, int tile,
+                                            uint32_t skip_models, const uint32_t *list, uint32_t n,
+                                            uint32_t n_l, int tile,
                                             long long b, uint32_t *acc, uint32_t *stage, uint32_t *cnt,
                                             int lane, DevStatus *st)
 {
-    const uint32_t idx = static_cast<uint32_t>(tile) * 32u + static_cast<uint32_t>(lane);
-    const bool listed = idx < n;
+    // tiles [0, tiles_h) cover the heavy entries list[0, n_h); the rest cover
+    // the light entries list[P - n_l, P)
+    const uint32_t n_h = n & 0xFFFFFFFFu;
+    const uint32_t tiles_h = (n_h + 31u) >> 5;
+    uint32_t idx;
+    bool listed;
+    if (static_cast<uint32_t>(tile) < tiles_h) {
+        idx = static_cast<uint32_t>(tile) * 32u + static_cast<uint32_t>(lane);
+        listed = idx < n_h;
+    } else {
+        idx = static_cast<uint32_t>(v.P) - n_l + (static_cast<uint32_t>(tile) - tiles_h) * 32u +
+              static_cast<uint32_t>(lane);
+        listed = idx < static_cast<uint32_t>(v.P);
+    }
     const uint32_t e = listed ? __ldg(list + idx) : 0u;
     const int p = static_cast<int>(e & 0x7FFFFFFFu);
     const bool neg = DELTA && (e >> 31) != 0u;
@@ -1000,8 +1032,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     if (threadIdx.x < 2)
         s_cnt[threadIdx.x] = 0u;
 
-    const uint32_t n = __ldg(count);
-    const long long tiles = (n + 31u) >> 5;
+    const uint32_t n = __ldg(count);          // heavy entries, list[0, n)
+    const uint32_t n_l = __ldg(count + 1);    // light entries, list[P - n_l, P)
+    const long long tiles = ((n + 31u) >> 5) + ((n_l + 31u) >> 5);
     const long long total = rows * tiles;
     // tasks per CTA range: up to one per warp, fewer when that spreads the work
     // over more SMs, and few enough that a range touches at most kMaxSlots rows
@@ -1023,7 +1056,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
         if (warp < WARPS && task < total) {
             const long long row = task / tiles;
             const int tile = static_cast<int>(task - row * tiles);
-            decode_task<W, DELTA>(v, s_dec, s_skip, skip_models, list, n, tile, row * stride,
+            decode_task<W, DELTA>(v, s_dec, s_skip, skip_models, list, n, n_l, tile, row * stride,
                                   s_acc + (row - row0) * kScans, s_stage + warp * 16, s_cnt, lane, st);
         }
         __syncthreads();
@@ -1182,16 +1215,16 @@ cudaError_t launch_generate(void *out, int bits, uint64_t seed, int64_t scan0, i
 }
 
 cudaError_t launch_enc_streams(const void *counts, int w, int P, int nblk, Tables tb, uint4 *desc, uint32_t *slots,
-                               unsigned long long *stats, cudaStream_t st)
+                               unsigned long long *stats, uint8_t *pclass, cudaStream_t st)
 {
     const long long total = static_cast<long long>(nblk) * P;
     const unsigned grid = static_cast<unsigned>((total + kEncThreads - 1) / kEncThreads);
     if (w == 1)
         k_enc_streams<uint8_t><<<grid, kEncThreads, 0, st>>>(static_cast<const uint8_t *>(counts), P, nblk, tb,
-                                                             desc, slots, stats);
+                                                             desc, slots, stats, pclass);
     else
         k_enc_streams<uint16_t><<<grid, kEncThreads, 0, st>>>(static_cast<const uint16_t *>(counts), P, nblk, tb,
-                                                              desc, slots, stats);
+                                                              desc, slots, stats, pclass);
     return cudaGetLastError();
 }
 
@@ -1216,18 +1249,18 @@ cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const
     return cudaGetLastError();
 }
 
-cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, uint8_t *base_mask, int P, int mode,
-                        uint32_t *list, uint32_t *count, void *out, const void *base_img, long long n_elems,
-                        int out_bytes, cudaStream_t st)
+cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t *pclass, uint8_t *base_mask,
+                        int P, int mode, uint32_t *list, uint32_t *count, void *out, const void *base_img,
+                        long long n_elems, int out_bytes, cudaStream_t st)
 {
     const long long n_vec = n_elems * out_bytes / 16;
     const int n_list = (P + kPlanThreads - 1) / kPlanThreads;
     int fill = static_cast<int>((n_vec + kPlanThreads * 4 - 1) / (kPlanThreads * 4));
     fill = fill < 1 ? 1 : (fill > 8 * sm_count() ? 8 * sm_count() : fill);
-    cudaError_t e = cudaMemsetAsync(count, 0, sizeof(uint32_t), st);
+    cudaError_t e = cudaMemsetAsync(count, 0, 2 * sizeof(uint32_t), st);
     if (e != cudaSuccess)
         return e;
-    k_plan<<<n_list + fill, kPlanThreads, 0, st>>>(mask, valid, base_mask, P, mode, n_list, list, count,
+    k_plan<<<n_list + fill, kPlanThreads, 0, st>>>(mask, valid, pclass, base_mask, P, mode, n_list, list, count,
                                                    static_cast<uint4 *>(out), static_cast<const uint4 *>(base_img),
                                                    n_vec);
     return cudaGetLastError();

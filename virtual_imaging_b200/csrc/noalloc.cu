@@ -16,7 +16,8 @@ constexpr int kMaxPixels = QEM_NOALLOC_MAX_PIXELS;
 constexpr int kMaxDevices = 64;
 constexpr int kPlanThreads = 1024;
 
-// Layout of the fixed working memory: error status, list length, listed pixels.
+// Layout of the fixed working memory: error status, list length (count, then
+// reserved[0] = 0 as the decoder's second list segment), listed pixels.
 struct Scratch {
     DevStatus status;
     uint32_t count;
@@ -95,8 +96,10 @@ __global__ void __launch_bounds__(kPlanThreads) k_noalloc_plan(const uint8_t *__
             base += s_total;
             __syncthreads();
         }
-        if (threadIdx.x == 0)
+        if (threadIdx.x == 0) {
             s->count = base;
+            s->reserved[0] = 0u;     // no light-class entries: the whole list is one segment
+        }
         return;
     }
     const long long stride = static_cast<long long>(gridDim.x - 1) * blockDim.x;

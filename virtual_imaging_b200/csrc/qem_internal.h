@@ -106,18 +106,21 @@ cudaError_t launch_generate(void *out, int bits, uint64_t seed, int64_t scan0, i
 
 cudaError_t launch_enc_streams(const void *counts, int w, int P, int nblk, Tables tb,
                                uint4 *desc, uint32_t *slots, unsigned long long *stats,
-                               cudaStream_t st);
+                               uint8_t *pclass, cudaStream_t st);
 cudaError_t launch_enc_layout(uint4 *desc, int P, int G, int nblk, uint32_t *groups,
                               uint32_t *blk_len, cudaStream_t st);
 cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const uint4 *desc,
                                const uint32_t *slots, const unsigned long long *blk_dst,
                                cudaStream_t st);
 
-// plan: builds the signed pixel list (CTA 0) and initialises the output rows
-// (other CTAs): mode 0 = full query (out = 0), 1 = delta (out = baseline image)
-cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, uint8_t *base_mask, int P,
-                        int mode, uint32_t *list, uint32_t *count, void *out,
-                        const void *base_img, long long n_elems, int out_bytes,
+// decode_reduce reads count[0] heavy entries from list[0..) and count[1]
+// light entries from list[P - count[1], P).
+// plan: builds the signed pixel list, heavy class from the front (count[0]),
+// light class from the back (count[1]), and initialises the output rows:
+// mode 0 = full query (out = 0), 1 = delta (out = baseline image)
+cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t *pclass,
+                        uint8_t *base_mask, int P, int mode, uint32_t *list, uint32_t *count,
+                        void *out, const void *base_img, long long n_elems, int out_bytes,
                         cudaStream_t st);
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count,
                                  int stride, long long rows, void *out, int out_bytes,
