@@ -45,8 +45,9 @@ __device__ __forceinline__ void report(DevStatus *st, uint32_t flag, long long b
 // running off the end; the caller's length checks then reject it.
 struct Bits {
     const uint32_t *first;
-    uint32_t wi;     // next word to load
+    uint32_t wi;     // index of the next word to enter the reservoir
     uint32_t li;     // last word that may be loaded
+    uint32_t nx;     // that next word, loaded one top-up ahead
     uint32_t lo, hi;
     int n;
     int lead;        // bits of the first word before the stream start
@@ -62,13 +63,16 @@ struct Bits {
         hi = 0u;
         n = 32 - lead;
         wi = 1u;
+        nx = __ldg(first + min(1u, li));
     }
-    // requires n < 32
+    // requires n < 32; the word it adds was loaded by the previous top-up, and
+    // the load for the following one is issued here
     __device__ __forceinline__ void refill()
     {
-        const uint32_t w = __ldg(first + min(wi, li));
+        const uint32_t w = nx;
+        nx = __ldg(first + min(wi + 1u, li));
         lo |= w << n;
-        hi |= n ? (w >> (32 - n)) : 0u;
+        hi |= __funnelshift_l(w, 0u, n);
         n += 32;
         ++wi;
     }
