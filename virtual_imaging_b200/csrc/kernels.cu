@@ -47,7 +47,8 @@ struct Bits {
     const uint32_t *first;
     uint32_t wi;     // index of the next word to enter the reservoir
     uint32_t li;     // last word that may be loaded
-    uint32_t nx;     // that next word, loaded one top-up ahead
+    uint32_t nx0;    // words wi and wi + 1, loaded two top-ups ahead
+    uint32_t nx1;
     uint32_t lo, hi;
     int n;
     int lead;        // bits of the first word before the stream start
@@ -63,14 +64,16 @@ struct Bits {
         hi = 0u;
         n = 32 - lead;
         wi = 1u;
-        nx = __ldg(first + min(1u, li));
+        nx0 = __ldg(first + min(1u, li));
+        nx1 = __ldg(first + min(2u, li));
     }
-    // requires n < 32; the word it adds was loaded by the previous top-up, and
-    // the load for the following one is issued here
+    // requires n < 32; the word it adds was loaded two top-ups earlier, and
+    // the load for the one after next is issued here
     __device__ __forceinline__ void refill()
     {
-        const uint32_t w = nx;
-        nx = __ldg(first + min(wi + 1u, li));
+        const uint32_t w = nx0;
+        nx0 = nx1;
+        nx1 = __ldg(first + min(wi + 2u, li));
         lo |= w << n;
         hi |= __funnelshift_l(w, 0u, n);
         n += 32;
@@ -1306,8 +1309,8 @@ cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const 
                                  cudaStream_t st, bool delta)
 {
     if (v.w == 1)
-        return delta ? launch_dr<1, 1024, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
-                     : launch_dr<1, 1024, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
+        return delta ? launch_dr<1, 768, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
+                     : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
     return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
                  : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
 }
