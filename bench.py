@@ -254,6 +254,16 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_encode(dev, torch, V):
+    """Bounded encode case for ncu: the default geometry (192x192 uint8, same counts) but 16
+    blocks (302 MB of raw counts, above the 126 MB L2), generated and encoded once."""
+    w = W.workload("c4")
+    w.scan_rows = 16
+    res, buf, t_enc = build_resident(w, dev, torch, V)
+    print(json.dumps({"encode_s": t_enc, "blocks": w.n_blocks}), flush=True)
+    res.free()
+
+
 def run_profile_case(dev, torch, V):
     """Small bounded case for ncu: build the default resident, then a few bright-field / annular
     block_stride-1 queries (the kernels ncu captures are the k_decode_reduce launches)."""
@@ -279,12 +289,13 @@ def run_profile_case(dev, torch, V):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="c4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true", help="bounded case for ncu captures")
+    ap.add_argument("--profile-encode", action="store_true", help="bounded encode case for ncu captures")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -309,12 +320,17 @@ def main():
     if args.profile:
         run_profile_case(dev, torch, V)
         return
+    if args.profile_encode:
+        run_profile_encode(dev, torch, V)
+        return
     w = W.workload(args.config)
     res, buf, _ = build_resident(w, dev, torch, V)
     # a second, warm encode of the same counts for the encode figure (chunked workloads keep the first)
     enc_s = None
+    enc_prof = None
     if buf.shape[0] == w.n_scans:
         res2 = V.Resident.create((w.scan_rows, w.scan_cols), (w.det_rows, w.det_cols), w.dtype_bits)
+        res2.profile(True)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -322,6 +338,7 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         enc_s = e0.elapsed_time(e1) / 1e3
+        enc_prof = {k: round(v[1], 3) for k, v in res2.profile_read().items() if v[0]}
         res2.free()
     # block decode leg (16 blocks)
     nd = min(16, w.n_blocks)
@@ -456,7 +473,7 @@ def main():
                         "enc_gbs": round(v["enc_gbs"], 1), "hbm_frac_enc": round(v["enc_gbs"] / hbm, 4)}
                     for k, v in per_query.items()},
         "kernels_ms_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[0]},
-        "encode": {"gbs_raw": (w.raw_bytes / enc_s / 1e9) if enc_s else None, "s": enc_s,
+        "encode": {"gbs_raw": (w.raw_bytes / enc_s / 1e9) if enc_s else None, "s": enc_s, "kernels_ms": enc_prof,
                    "hbm_frac": ((w.raw_bytes + info["payload_bytes"] + info["group_bytes"]) / enc_s / 1e9 / hbm)
                    if enc_s else None},
         "decode_blocks": {"blocks": nd, "s": dec_s, "gcounts_per_s": nd * 512 * w.n_pixels / dec_s / 1e9,

@@ -410,11 +410,19 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
         const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
 
         uint32_t nnz = 0, mn = 0xFFFFFFFFu, mx = 0;
+        uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;      // first four nonzeros: scan | value << 16
         {
             const T *q = col;
 #pragma unroll 8
             for (int i = 0; i < kScans; ++i, q += P) {
                 const uint32_t v = *q;
+                if (v && nnz < 4u) {
+                    const uint32_t e = static_cast<uint32_t>(i) | (v << 16);
+                    c0 = nnz == 0u ? e : c0;
+                    c1 = nnz == 1u ? e : c1;
+                    c2 = nnz == 2u ? e : c2;
+                    c3 = nnz == 3u ? e : c3;
+                }
                 nnz += v != 0u;
                 mn = min(mn, v);
                 mx = max(mx, v);
@@ -503,6 +511,19 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
             }
             if (nacc > 0)
                 slot[wi] = static_cast<uint32_t>(acc << (32 - nacc));
+            {
+                // move the section (bits [32*kSlotWords - T, 32*kSlotWords) of the
+                // slot) down to bit 0, zero-filled above its end, so that the
+                // compaction copies plain bytes
+                const int o0 = 32 * kSlotWords - static_cast<int>(Tbits);
+                const int w0 = o0 >> 5, sh = o0 & 31;
+                const int nw = static_cast<int>((Tbits + 31u) >> 5);
+                for (int i = 0; i < nw; ++i) {
+                    const uint32_t a = slot[w0 + i];
+                    const uint32_t c = w0 + i + 1 < kSlotWords ? slot[w0 + i + 1] : 0u;
+                    slot[i] = __funnelshift_r(a, c, sh);
+                }
+            }
 
             const uint32_t paired = 2u + has_base * W + 64u * static_cast<uint32_t>(shift) + (Tbits + 7u) / 8u;
             uint32_t size;
@@ -524,6 +545,50 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
             else
                 d.y = static_cast<uint32_t>(form);
             d.z = base | (nnz << 16);
+            if (form == kSparse && size - 2u <= static_cast<uint32_t>(kSlotWords) * 4u) {
+                // the column is hot in L1 now: write the sparse payload (n-1,
+                // 9-bit positions, values) into the slot for the compaction to copy
+                uint8_t *o = reinterpret_cast<uint8_t *>(slot);
+                uint32_t k = 0, acc = 0;
+                int nacc = 0;
+                o[k++] = static_cast<uint8_t>(nnz - 1u);
+                auto put_pos = [&](uint32_t i) {
+                    acc |= i << nacc;
+                    nacc += 9;
+                    while (nacc >= 8) {
+                        o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                        acc >>= 8;
+                        nacc -= 8;
+                    }
+                };
+                auto put_val = [&](uint32_t v) {
+                    o[k++] = static_cast<uint8_t>(v & 0xFFu);
+                    if (W == 2)
+                        o[k++] = static_cast<uint8_t>(v >> 8);
+                };
+                if (nnz <= 4u) {
+                    // the first pass kept them: no further reads
+                    const uint32_t c[4] = {c0, c1, c2, c3};
+                    for (uint32_t j = 0; j < nnz; ++j)
+                        put_pos(c[j] & 0xFFFFu);
+                    if (nacc > 0)
+                        o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                    for (uint32_t j = 0; j < nnz; ++j)
+                        put_val(c[j] >> 16);
+                } else {
+                    const T *q = col;
+                    for (int i = 0; i < kScans; ++i, q += P)
+                        if (*q)
+                            put_pos(static_cast<uint32_t>(i));
+                    if (nacc > 0)
+                        o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                    q = col;
+                    for (int i = 0; i < kScans; ++i, q += P)
+                        if (*q)
+                            put_val(*q);
+                }
+                d.y |= 1u << 16;          // the payload after the header is in the slot
+            }
         }
         desc[sid] = d;
         if (pclass && b == 0) {
@@ -578,6 +643,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t x, uint32_t *s
 
 // a4 (first half): per block, exclusive scan of stream lengths in pixel order
 // -> per-stream offsets (desc.w), block length, and the group records (S1).
+// Each warp scans one contiguous chunk of pixels 32 at a time (coalesced
+// descriptor reads and writes); a block-wide scan joins the chunks; then
+// each warp writes whole group records (lane j holds stream j's end).
 __global__ void __launch_bounds__(kLayoutThreads) k_enc_layout(uint4 *__restrict__ desc, int P, int G,
                                                               uint32_t *__restrict__ groups,
                                                               uint32_t *__restrict__ blk_len)
@@ -585,60 +653,59 @@ __global__ void __launch_bounds__(kLayoutThreads) k_enc_layout(uint4 *__restrict
     __shared__ uint32_t s_warp[32];
     const int b = blockIdx.x;
     uint4 *d = desc + static_cast<size_t>(b) * P;
-    const int per = (P + kLayoutThreads - 1) / kLayoutThreads;
-    const int p0 = min(P, static_cast<int>(threadIdx.x) * per);
-    const int p1 = min(P, p0 + per);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = kLayoutThreads / 32;
+    const int chunk = ((P + NW - 1) / NW + 31) & ~31;
+    const int c0 = min(P, warp * chunk), c1 = min(P, c0 + chunk);
     uint32_t local = 0;
-    for (int p = p0; p < p1; ++p)
+    for (int p = c0 + lane; p < c1; p += 32)
         local += d[p].x;
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        local += __shfl_xor_sync(kFull, local, o);
     uint32_t total;
-    uint32_t run = block_exclusive_scan(local, s_warp, total);
-    for (int p = p0; p < p1; ++p) {
-        d[p].w = run;
-        run += d[p].x;
+    const uint32_t mine = lane == 0 ? local : 0u;
+    uint32_t run = __shfl_sync(kFull, block_exclusive_scan(mine, s_warp, total), 0);
+    for (int base = c0; base < c1; base += 32) {
+        const int p = base + lane;
+        const uint32_t len = p < c1 ? d[p].x : 0u;
+        uint32_t inc = len;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o)
+                inc += y;
+        }
+        if (p < c1)
+            d[p].w = run + inc - len;
+        run += __shfl_sync(kFull, inc, 31);
     }
     if (threadIdx.x == 0)
         blk_len[b] = total;
     __syncthreads();
     uint32_t *gb = groups + static_cast<size_t>(b) * G * kGroupWords;
-    for (int g = threadIdx.x; g < G; g += kLayoutThreads) {
-        uint32_t *rec = gb + static_cast<size_t>(g) * kGroupWords;
+    for (int g = warp; g < G; g += NW) {
+        const int p = 32 * g + lane;
         const uint32_t base = d[32 * g].w;
-        rec[0] = base;
-        uint32_t end = 0;
-        for (int j = 0; j < 32; j += 2) {
-            uint32_t lo, hi;
-            const int pa = 32 * g + j;
-            if (pa < P)
-                end = d[pa].w + d[pa].x - base;
-            lo = end;
-            if (pa + 1 < P)
-                end = d[pa + 1].w + d[pa + 1].x - base;
-            hi = end;
-            rec[1 + j / 2] = lo | (hi << 16);
-        }
+        // the last real stream's end repeats over the padding lanes of the last group
+        const int q = min(p, P - 1);
+        const uint4 dq = d[q];
+        const uint32_t end = dq.w + dq.x - base;
+        const uint32_t other = __shfl_down_sync(kFull, end, 1);
+        uint32_t *rec = gb + static_cast<size_t>(g) * kGroupWords;
+        if (lane == 0)
+            rec[0] = base;
+        if ((lane & 1) == 0)
+            rec[1 + lane / 2] = end | (other << 16);
     }
 }
 
-// a4 (second half): write every stream's bytes at blk_dst[b] + offset.
+// Write one stream's bytes (header and form payload, spec S2/S3) at o.
 template <typename T>
-__global__ void __launch_bounds__(256) k_enc_compact(const T *__restrict__ counts, int P, int nblk,
-                                                    const uint4 *__restrict__ desc,
-                                                    const uint32_t *__restrict__ slots,
-                                                    const unsigned long long *__restrict__ blk_dst)
+__device__ __forceinline__ void write_stream(uint8_t *o, const T *col, int P, const uint4 d, const uint32_t *sl)
 {
     constexpr uint32_t W = sizeof(T);
-    const long long sid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (sid >= static_cast<long long>(nblk) * P)
-        return;
-    const uint4 d = desc[sid];
-    if (d.x == 0u)
-        return;
-    const int b = static_cast<int>(sid / P);
-    const int p = static_cast<int>(sid - static_cast<long long>(b) * P);
-    const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
-    uint8_t *o = reinterpret_cast<uint8_t *>(blk_dst[b]) + d.w;
-    const uint32_t hdr = d.y & 0xFFFFu;
+    const uint32_t hdr = d.y & 0xFFFFu;     // (bits 16+ of d.y: T for paired, a flag for sparse)
     const int form = static_cast<int>(hdr & 7u);
     o[0] = static_cast<uint8_t>(hdr & 0xFFu);
     o[1] = static_cast<uint8_t>(hdr >> 8);
@@ -654,6 +721,17 @@ __global__ void __launch_bounds__(256) k_enc_compact(const T *__restrict__ count
         const T *q = col;
         for (int i = 0; i < kScans; ++i, q += P)
             put(*q);
+    } else if (form == kSparse && ((d.y >> 16) & 1u)) {
+        const int nbytes = static_cast<int>(d.x) - 2;
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(sl);
+        for (int q = 0; q < nbytes; q += 16) {
+            const uint4 c = __ldcs(s4 + q / 16);
+            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (q + i < nbytes)
+                    o[k + q + i] = static_cast<uint8_t>(wv[i >> 2] >> (8 * (i & 3)));
+        }
     } else if (form == kSparse) {
         const uint32_t nnz = d.z >> 16;
         o[k++] = static_cast<uint8_t>(nnz - 1u);
@@ -697,16 +775,72 @@ __global__ void __launch_bounds__(256) k_enc_compact(const T *__restrict__ count
                 }
             }
         }
+        // the tANS section starts at byte 0 of the stream's 16-byte aligned
+        // slot: independent 16-byte loads, then bytes
         const uint32_t Tbits = d.y >> 16;
-        const uint32_t *sl = slots + static_cast<size_t>(sid) * kSlotWords;
         const int nbytes = static_cast<int>((Tbits + 7u) / 8u);
-        const int o0 = 32 * kSlotWords - static_cast<int>(Tbits);
-        for (int q = 0; q < nbytes; ++q) {
-            const int bp = o0 + 8 * q;
-            const int wi = bp >> 5;
-            const uint64_t x = static_cast<uint64_t>(sl[wi]) |
-                               (wi + 1 < kSlotWords ? static_cast<uint64_t>(sl[wi + 1]) << 32 : 0ull);
-            o[k++] = static_cast<uint8_t>((x >> (bp & 31)) & 0xFFu);
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(sl);
+        for (int q = 0; q < nbytes; q += 16) {
+            const uint4 c = __ldcs(s4 + q / 16);
+            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (q + i < nbytes)
+                    o[k + q + i] = static_cast<uint8_t>(wv[i >> 2] >> (8 * (i & 3)));
+        }
+    }
+}
+
+constexpr int kCompactThreads = 128;
+constexpr int kCompactBytes = 64 * 1024;   // staged byte range per CTA (dynamic shared memory)
+
+// a4 (second half): write every stream's bytes at blk_dst[b] + offset.  A CTA
+// takes 128 consecutive pixels of one block, whose streams are contiguous in
+// the payload; when their byte range fits, each thread writes its stream into
+// shared memory (placed congruent to the destination modulo 16) and the CTA
+// stores the range with aligned 16-byte writes, bytes only at the two ragged
+// ends.  Larger ranges (incompressible data) are written in place.
+template <typename T>
+__global__ void __launch_bounds__(kCompactThreads) k_enc_compact(const T *__restrict__ counts, int P, int nblk,
+                                                                const uint4 *__restrict__ desc,
+                                                                const uint32_t *__restrict__ slots,
+                                                                const unsigned long long *__restrict__ blk_dst)
+{
+    extern __shared__ __align__(16) uint8_t s_buf[];     // kCompactBytes + 32
+    const int b = blockIdx.y;
+    const int p0 = blockIdx.x * kCompactThreads;
+    const int p1 = min(P, p0 + kCompactThreads);
+    const int p = p0 + static_cast<int>(threadIdx.x);
+    const long long sid = static_cast<long long>(b) * P + p;
+    uint8_t *blk = reinterpret_cast<uint8_t *>(blk_dst[b]);
+    const uint4 first = desc[static_cast<long long>(b) * P + p0];
+    const uint4 last = desc[static_cast<long long>(b) * P + p1 - 1];
+    const uint32_t r0 = first.w, r1 = last.w + last.x;         // the CTA's byte range in the block
+    const bool staged = r1 - r0 <= static_cast<uint32_t>(kCompactBytes);
+    uint8_t *dst0 = blk + r0;
+    const uint32_t mis = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(dst0) & 15u);
+    if (p < p1) {
+        const uint4 d = desc[sid];
+        if (d.x) {
+            const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
+            uint8_t *o = staged ? s_buf + mis + (d.w - r0) : blk + d.w;
+            write_stream<T>(o, col, P, d, slots + static_cast<size_t>(sid) * kSlotWords);
+        }
+    }
+    if (!staged)
+        return;
+    __syncthreads();
+    const uint32_t len = r1 - r0;
+    const uint32_t span = mis + len;                            // staged bytes from the aligned start
+    uint8_t *aligned = dst0 - mis;
+    for (uint32_t c = threadIdx.x; c * 16 < span; c += kCompactThreads) {
+        const uint32_t lo = c * 16, hi = lo + 16;
+        if (lo >= mis && hi <= span) {
+            *reinterpret_cast<uint4 *>(aligned + lo) = *reinterpret_cast<const uint4 *>(s_buf + lo);
+        } else {
+            for (uint32_t i = lo; i < hi && i < span; ++i)
+                if (i >= mis)
+                    aligned[i] = s_buf[i];
         }
     }
 }
@@ -1245,14 +1379,23 @@ cudaError_t launch_enc_layout(uint4 *desc, int P, int G, int nblk, uint32_t *gro
 cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const uint4 *desc,
                                const uint32_t *slots, const unsigned long long *blk_dst, cudaStream_t st)
 {
-    const long long total = static_cast<long long>(nblk) * P;
-    const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+    const dim3 grid((P + kCompactThreads - 1) / kCompactThreads, nblk);
+    const int smem = kCompactBytes + 32;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(k_enc_compact<uint8_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_enc_compact<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return e;
+        attr = true;
+    }
     if (w == 1)
-        k_enc_compact<uint8_t><<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(counts), P, nblk, desc, slots,
-                                                     blk_dst);
+        k_enc_compact<uint8_t><<<grid, kCompactThreads, smem, st>>>(static_cast<const uint8_t *>(counts), P, nblk,
+                                                                     desc, slots, blk_dst);
     else
-        k_enc_compact<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(counts), P, nblk, desc,
-                                                      slots, blk_dst);
+        k_enc_compact<uint16_t><<<grid, kCompactThreads, smem, st>>>(static_cast<const uint16_t *>(counts), P, nblk,
+                                                                      desc, slots, blk_dst);
     return cudaGetLastError();
 }
 

@@ -17,7 +17,7 @@ constexpr int kPairs = 256;        // consecutive count pairs per stream
 constexpr int kStates = 1024;      // tANS states (page: 1024-state table)
 constexpr int kModels = 32;        // Poisson pair models (page: 32)
 constexpr int kGroupWords = 17;    // 1 x u32 base + 32 x u16 relative ends (spec S1)
-constexpr int kSlotWords = 82;     // per-stream tANS scratch: ceil((10 + 256*10)/32) + 1 words
+constexpr int kSlotWords = 84;     // per-stream tANS scratch: >= ceil((10 + 256*10)/32) + 1 words, 16-byte multiple
 constexpr int kArenaPad = 64;      // zero bytes after the last block of an arena
 
 enum Form : int { kEmpty = 0, kConstant = 1, kSparse = 2, kPaired = 3, kLiteral = 4 };
