@@ -41,7 +41,8 @@ typedef enum {
                                malformed stream -> error, the result is not returned) */
     QEM_ERR_CUDA = 3,       /* a CUDA runtime call failed                            */
     QEM_ERR_OOM = 4,        /* device allocation failed                              */
-    QEM_ERR_TIMEOUT = 5,    /* a bounded host wait on the device ran out             */
+    QEM_ERR_TIMEOUT = 5,    /* a bounded wait ran out (host on the device, or a
+                               kernel on its shared-memory table copy)             */
     QEM_ERR_TAINTED = 6,    /* delta refused: the stride's baseline was invalidated by
                                a failed decode (page "Contract", queued queries)      */
     QEM_ERR_STATE = 7       /* call not valid in the resident's current state         */
@@ -67,7 +68,9 @@ typedef struct {
 } qem_info_t;
 
 /* Per-kernel device time, gathered with CUDA events on the launching stream
- * while profiling is enabled (qem_profile). */
+ * while profiling is enabled (qem_profile).  A masked sum launches the plan
+ * and decode_reduce kernels; the slot QEM_K_FINALIZE is kept for layout and
+ * stays at zero (the decode updates the kept baseline image itself). */
 typedef struct {
     int64_t launches[8];
     double ms[8];

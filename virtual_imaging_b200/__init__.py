@@ -209,6 +209,8 @@ class Resident:
     # ---- queries ---------------------------------------------------------------
     def _query(self, fn, name, mask, block_stride, out_bits, out, wait, stream):
         if out is None:
+            if block_stride < 1:
+                raise QemError(QEM_ERR_ARG, name)
             n_blocks, _, _, auto = self._static()
             rows = -(-n_blocks // block_stride)
             bits = auto if out_bits == 0 else out_bits

@@ -77,7 +77,8 @@ struct qem_resident {
     size_t pinned_blocks = 0;
 
     uint32_t *d_list = nullptr;
-    uint32_t *d_count = nullptr;
+    uint32_t *d_count = nullptr;                // two (heavy, light) counter pairs, used in turn
+    int count_pair = 0;                         // the pair the next query fills
     DevStatus *d_status = nullptr;
     DevStatus *h_status = nullptr;              // pinned
     std::map<int, Baseline> baselines;
@@ -262,6 +263,8 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
         (rc = dalloc(&r->d_list, size_t(r->P) * 4)) || (rc = dalloc(&r->d_count, 16)) ||
         (rc = dalloc(&r->d_status, sizeof(DevStatus))))
         return fail(rc);
+    if (cudaMemset(r->d_count, 0, 16) != cudaSuccess)
+        return fail(QEM_ERR_CUDA);
     if (cudaMallocHost(&r->h_status, sizeof(DevStatus)) != cudaSuccess)
         return fail(QEM_ERR_OOM);
     std::memset(r->h_status, 0, sizeof(DevStatus));
@@ -375,13 +378,14 @@ int report_errors(qem_resident *r, cudaStream_t st)
             kv.second.state = kTainted;
             kv.second.pending = false;
         }
+    const bool timed_out = (r->h_status->flags & kErrWait) != 0u;
     const unsigned long long rows = r->h_status->rows, streams = r->h_status->streams;
     std::memset(r->h_status, 0, sizeof(DevStatus));
     r->h_status->rows = rows;
     r->h_status->streams = streams;
     QEM_CK(cudaMemcpyAsync(r->d_status, r->h_status, sizeof(DevStatus), cudaMemcpyHostToDevice, st));
     QEM_CK(cudaStreamSynchronize(st));
-    return QEM_ERR_MALFORMED;
+    return timed_out ? QEM_ERR_TIMEOUT : QEM_ERR_MALFORMED;
 }
 
 int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, void *d_out, int32_t *used,
@@ -402,7 +406,6 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         return QEM_ERR_ARG;
     const long long rows = (r->B + k - 1) / k;
     const long long n_elems = rows * kScans;
-    const size_t out_bytes = static_cast<size_t>(n_elems) * (bits / 8);
 
     Baseline &bl = r->baselines[k];
     if (!bl.d_mask) {
@@ -418,19 +421,21 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         if (bl.state == kValid && bl.out_bits == bits)
             mode = 1;
     }
+    uint32_t *count = r->d_count + 2 * r->count_pair;
+    uint32_t *count_next = r->d_count + 2 * (r->count_pair ^ 1);
     int rc = timed(r, QEM_K_PLAN, st, [&] {
-        return launch_plan(d_mask, r->d_valid, r->d_pclass, bl.d_mask, r->P, mode, r->d_list, r->d_count, d_out,
-                           bl.d_img, n_elems, bits / 8, st);
+        return launch_plan(d_mask, r->d_valid, r->d_pclass, bl.d_mask, r->P, mode, r->d_list, count, count_next,
+                           d_out, bl.d_img, n_elems, bits / 8, st);
     });
     if (rc)
         return rc;
+    r->count_pair ^= 1;
+    // the decode adds every term to d_out and to the stride's kept image, so
+    // the kept image is this query's result without a copy
     rc = timed(r, QEM_K_DECODE_REDUCE, st, [&] {
-        return launch_decode_reduce(r->view(), r->tables(), r->d_list, r->d_count, k, rows, d_out, bits / 8,
-                                    r->d_status, r->n_sm, st, mode == 1);
+        return launch_decode_reduce(r->view(), r->tables(), r->d_list, count, k, rows, d_out, bits / 8,
+                                    r->d_status, r->n_sm, st, mode == 1, bl.d_img);
     });
-    if (rc)
-        return rc;
-    rc = timed(r, QEM_K_FINALIZE, st, [&] { return launch_copy(bl.d_img, d_out, out_bytes, st); });
     if (rc)
         return rc;
     bl.state = kValid;

@@ -37,6 +37,50 @@ __device__ __forceinline__ void report(DevStatus *st, uint32_t flag, long long b
     }
 }
 
+// Shared-memory tables arrive by the bulk-copy engine: one thread starts the
+// copies, which complete on an mbarrier; every thread waits on it before its
+// first table read, so the copy overlaps the CTA's setup and its first stream
+// opens.  The wait is bounded: past kWaitLimit polls it flags kErrWait and
+// returns false (the query then reports an error instead of a result).
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+__device__ __forceinline__ void tables_start(uint64_t *bar, void *s_dst0, const void *g_src0, uint32_t bytes0,
+                                             void *s_dst1, const void *g_src1, uint32_t bytes1)
+{
+    const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes0 + bytes1) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(s_dst0))),
+                 "l"(g_src0), "r"(bytes0), "r"(b)
+                 : "memory");
+    if (bytes1)
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(s_dst1))),
+                     "l"(g_src1), "r"(bytes1), "r"(b)
+                     : "memory");
+}
+
+__device__ __forceinline__ bool tables_wait(uint64_t *bar, DevStatus *st)
+{
+    const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done)
+                     : "r"(b)
+                     : "memory");
+        if (done)
+            return true;
+    }
+    atomicOr(&st->flags, kErrWait);
+    return false;
+}
+
 // Forward LSB-first bit reader over aligned 32-bit little-endian words: a
 // 64-bit reservoir (lo, hi) holding `n` valid bits.  Words are addressed by
 // index from `first` (the aligned word holding the stream's first byte), and
@@ -858,19 +902,28 @@ constexpr int kPlanThreads = 256;
 // Order inside a class does not matter to the sums (integer addition).
 // Full query: mask && valid; delta: pixels whose (mask && valid) changed
 // against the stored baseline mask, leaving pixels flagged in bit 31.  Every
-// thread then stores the new mask as the baseline.  Blocks past n_list_blocks
-// initialise the output rows (0, or the baseline image for a delta).
+// thread then stores the new mask as the baseline.  A block reserves its
+// list slots with one atomic per class.  Blocks past n_list_blocks initialise
+// the rows: a full query zeroes the output and the kept image, a delta starts
+// the output from the kept image (the decode adds its terms to both).  The
+// counter pair of the next query (count_next) is cleared here, so that no
+// separate clear is needed between queries.
 __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict__ mask,
                                                       const uint8_t *__restrict__ valid,
                                                       const uint8_t *__restrict__ pclass,
                                                       uint8_t *__restrict__ base_mask, int P, int mode,
                                                       int n_list_blocks, uint32_t *__restrict__ list,
-                                                      uint32_t *__restrict__ count, uint4 *__restrict__ out,
-                                                      const uint4 *__restrict__ base_img, long long n_vec)
+                                                      uint32_t *__restrict__ count,
+                                                      uint32_t *__restrict__ count_next, uint4 *__restrict__ out,
+                                                      uint4 *__restrict__ keep, long long n_vec)
 {
+    if (blockIdx.x == 0 && threadIdx.x < 2)
+        count_next[threadIdx.x] = 0u;
     if (static_cast<int>(blockIdx.x) < n_list_blocks) {
+        constexpr int NW = kPlanThreads / 32;
+        __shared__ uint32_t s_h[NW], s_l[NW], s_at[2];
         const int p = static_cast<int>(blockIdx.x) * kPlanThreads + static_cast<int>(threadIdx.x);
-        const int lane = threadIdx.x & 31;
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
         bool emit = false, light = false;
         uint32_t entry = 0;
         uint8_t mk = 0;
@@ -891,31 +944,42 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
         }
         const unsigned bh = __ballot_sync(kFull, emit && !light);
         const unsigned bl = __ballot_sync(kFull, emit && light);
-        uint32_t at = 0;
-        if (lane == 0 && bh)
-            at = atomicAdd(count, static_cast<uint32_t>(__popc(bh)));
-        if (lane == 1 && bl)
-            at = atomicAdd(count + 1, static_cast<uint32_t>(__popc(bl)));
-        const uint32_t ah = __shfl_sync(kFull, at, 0);
-        const uint32_t al = __shfl_sync(kFull, at, 1);
+        if (lane == 0) {
+            s_h[warp] = static_cast<uint32_t>(__popc(bh));
+            s_l[warp] = static_cast<uint32_t>(__popc(bl));
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // exclusive prefix over the warps, then one reservation per class
+            uint32_t th = 0, tl = 0;
+            for (int w = 0; w < NW; ++w) {
+                const uint32_t a = s_h[w], c = s_l[w];
+                s_h[w] = th;
+                s_l[w] = tl;
+                th += a;
+                tl += c;
+            }
+            s_at[0] = th ? atomicAdd(count, th) : 0u;
+            s_at[1] = tl ? atomicAdd(count + 1, tl) : 0u;
+        }
+        __syncthreads();
         const unsigned below = (1u << lane) - 1u;
         if (emit && !light)
-            list[ah + __popc(bh & below)] = entry;
+            list[s_at[0] + s_h[warp] + __popc(bh & below)] = entry;
         if (emit && light)
-            list[P - 1 - (al + __popc(bl & below))] = entry;
+            list[P - 1 - (s_at[1] + s_l[warp] + __popc(bl & below))] = entry;
         return;
     }
     const long long stride = static_cast<long long>(gridDim.x - n_list_blocks) * blockDim.x;
     for (long long i = static_cast<long long>(blockIdx.x - n_list_blocks) * blockDim.x + threadIdx.x; i < n_vec;
-         i += stride)
-        out[i] = mode == 0 ? make_uint4(0u, 0u, 0u, 0u) : base_img[i];
-}
-
-__global__ void k_copy(uint4 *__restrict__ dst, const uint4 *__restrict__ src, long long n_vec)
-{
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_vec;
-         i += static_cast<long long>(gridDim.x) * blockDim.x)
-        dst[i] = src[i];
+         i += stride) {
+        if (mode == 0) {
+            out[i] = make_uint4(0u, 0u, 0u, 0u);
+            keep[i] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            out[i] = keep[i];
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -933,7 +997,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                                             uint32_t skip_models, const uint32_t *list, uint32_t n,
                                             uint32_t n_l, int tile,
                                             long long b, uint32_t *acc, uint32_t *stage, uint32_t *cnt,
-                                            int lane, DevStatus *st)
+                                            uint64_t *bar, bool &ready, int lane, DevStatus *st)
 {
     // tiles [0, tiles_h) cover the heavy entries list[0, n_h); the rest cover
     // the light entries list[P - n_l, P)
@@ -967,6 +1031,13 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
         ok = open_stream(S, W, b, p, st);
     if (!ok)
         S.form = kEmpty;
+    if (!ready) {
+        // first task of this thread: the tables must have landed (the stream
+        // opens above overlapped their copy)
+        if (!tables_wait(bar, st))
+            S.form = kEmpty;
+        ready = true;
+    }
 
     const unsigned nact = __popc(__ballot_sync(kFull, listed));
     if (lane == 0) {
@@ -1154,7 +1225,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
                                                              const uint32_t *__restrict__ list,
                                                              const uint32_t *__restrict__ count, int stride,
                                                              long long rows, void *__restrict__ out,
-                                                             int out_bytes, DevStatus *__restrict__ st)
+                                                             void *__restrict__ keep, int out_bytes,
+                                                             DevStatus *__restrict__ st)
 {
     constexpr int MAXW = THREADS / 32;
     // shared memory: decode tables of the 32 models | run tables of the first
@@ -1164,10 +1236,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     uint16_t *s_skip = reinterpret_cast<uint16_t *>(smem + kModels * kStates);
     uint32_t *s_stage = smem + kModels * kStates + skip_count * kStates / 2;   // 16 words per warp
     uint32_t *s_acc = s_stage + MAXW * 16;
-    for (int i = threadIdx.x; i < kModels * kStates / 4; i += THREADS)
-        reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
-    for (int i = threadIdx.x; i < skip_count * kStates / 8; i += THREADS)
-        reinterpret_cast<uint4 *>(s_skip)[i] = __ldg(reinterpret_cast<const uint4 *>(skip_g) + i);
+    __shared__ __align__(8) uint64_t s_bar;
+    if (threadIdx.x == 0)
+        tables_start(&s_bar, s_dec, dec_g, kModels * kStates * 4u, s_skip, skip_g,
+                     static_cast<uint32_t>(skip_count) * kStates * 2u);
+    bool ready = false;
     // per-CTA counters (rows, streams), added to the status once at the end
     __shared__ uint32_t s_cnt[2];
     if (threadIdx.x < 2)
@@ -1198,26 +1271,39 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
             const long long row = task / tiles;
             const int tile = static_cast<int>(task - row * tiles);
             decode_task<W, DELTA>(v, s_dec, s_skip, skip_models, list, n, n_l, tile, row * stride,
-                                  s_acc + (row - row0) * kScans, s_stage + warp * 16, s_cnt, lane, st);
+                                  s_acc + (row - row0) * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready,
+                                  lane, st);
         }
         __syncthreads();
         for (int i = threadIdx.x; i < nslot * kScans; i += THREADS) {
             const uint32_t val = s_acc[i];
             if (val) {
                 const long long o = (row0 + i / kScans) * kScans + (i % kScans);
-                if (out_bytes == 4)
+                if (out_bytes == 4) {
                     atomicAdd(reinterpret_cast<unsigned int *>(out) + o, val);
-                else
-                    atomicAdd(reinterpret_cast<unsigned long long *>(out) + o,
-                              static_cast<unsigned long long>(static_cast<long long>(static_cast<int>(val))));
+                    if (keep)
+                        atomicAdd(reinterpret_cast<unsigned int *>(keep) + o, val);
+                } else {
+                    const unsigned long long wide =
+                        static_cast<unsigned long long>(static_cast<long long>(static_cast<int>(val)));
+                    atomicAdd(reinterpret_cast<unsigned long long *>(out) + o, wide);
+                    if (keep)
+                        atomicAdd(reinterpret_cast<unsigned long long *>(keep) + o, wide);
+                }
             }
         }
         __syncthreads();
     }
     __syncthreads();
-    if (threadIdx.x == 0 && (s_cnt[0] | s_cnt[1])) {
-        atomicAdd(&st->rows, static_cast<unsigned long long>(s_cnt[0]));
-        atomicAdd(&st->streams, static_cast<unsigned long long>(s_cnt[1]));
+    if (threadIdx.x == 0) {
+        // a CTA leaves only after its table copy has landed (CTAs without
+        // tasks never waited on it)
+        if (!ready)
+            tables_wait(&s_bar, st);
+        if (s_cnt[0] | s_cnt[1]) {
+            atomicAdd(&st->rows, static_cast<unsigned long long>(s_cnt[0]));
+            atomicAdd(&st->streams, static_cast<unsigned long long>(s_cnt[1]));
+        }
     }
 }
 
@@ -1400,34 +1486,22 @@ cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const
 }
 
 cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t *pclass, uint8_t *base_mask,
-                        int P, int mode, uint32_t *list, uint32_t *count, void *out, const void *base_img,
-                        long long n_elems, int out_bytes, cudaStream_t st)
+                        int P, int mode, uint32_t *list, uint32_t *count, uint32_t *count_next, void *out,
+                        void *keep, long long n_elems, int out_bytes, cudaStream_t st)
 {
     const long long n_vec = n_elems * out_bytes / 16;
     const int n_list = (P + kPlanThreads - 1) / kPlanThreads;
     int fill = static_cast<int>((n_vec + kPlanThreads * 4 - 1) / (kPlanThreads * 4));
     fill = fill < 1 ? 1 : (fill > 8 * sm_count() ? 8 * sm_count() : fill);
-    cudaError_t e = cudaMemsetAsync(count, 0, 2 * sizeof(uint32_t), st);
-    if (e != cudaSuccess)
-        return e;
     k_plan<<<n_list + fill, kPlanThreads, 0, st>>>(mask, valid, pclass, base_mask, P, mode, n_list, list, count,
-                                                   static_cast<uint4 *>(out), static_cast<const uint4 *>(base_img),
+                                                   count_next, static_cast<uint4 *>(out), static_cast<uint4 *>(keep),
                                                    n_vec);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_copy(void *dst, const void *src, size_t bytes, cudaStream_t st)
-{
-    const long long n_vec = static_cast<long long>(bytes / 16);
-    int grid = static_cast<int>((n_vec + 255) / 256);
-    grid = grid < 1 ? 1 : (grid > 4 * sm_count() ? 4 * sm_count() : grid);
-    k_copy<<<grid, 256, 0, st>>>(static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), n_vec);
     return cudaGetLastError();
 }
 
 template <int W, int TH, bool DELTA>
 cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride, long long rows,
-                      void *out, int out_bytes, DevStatus *status, int n_sm, cudaStream_t st)
+                      void *out, void *keep, int out_bytes, DevStatus *status, int n_sm, cudaStream_t st)
 {
     // the run-decoded models are a prefix 0..k-1 (their (0,0) share falls as lambda grows)
     const int skip_count = __builtin_popcount(tb.skip_models);
@@ -1443,19 +1517,20 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
         attr = smem;
     }
     k_decode_reduce<W, TH, DELTA><<<n_sm, TH, smem, st>>>(v, tb.dec, tb.skip, tb.skip_models, skip_count, list,
-                                                          count, stride, rows, out, out_bytes, status);
+                                                          count, stride, rows, out, keep, out_bytes, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride,
                                  long long rows, void *out, int out_bytes, DevStatus *status, int n_sm,
-                                 cudaStream_t st, bool delta)
+                                 cudaStream_t st, bool delta, void *keep)
 {
     if (v.w == 1)
-        return delta ? launch_dr<1, 768, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
-                     : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
-    return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st)
-                 : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, out_bytes, status, n_sm, st);
+        return delta ? launch_dr<1, 768, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm, st)
+                     : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm,
+                                                st);
+    return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm, st)
+                 : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm, st);
 }
 
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,

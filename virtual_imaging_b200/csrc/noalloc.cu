@@ -161,5 +161,7 @@ extern "C" int qem_masked_sum_noalloc(qem_resident *res, const uint8_t *d_mask, 
         e = cudaStreamSynchronize(st);
     if (e != cudaSuccess)
         return QEM_ERR_CUDA;
+    if (flags & kErrWait)
+        return QEM_ERR_TIMEOUT;
     return flags ? QEM_ERR_MALFORMED : QEM_OK;
 }

@@ -22,7 +22,8 @@ constexpr int kArenaPad = 64;      // zero bytes after the last block of an aren
 
 enum Form : int { kEmpty = 0, kConstant = 1, kSparse = 2, kPaired = 3, kLiteral = 4 };
 
-// device status flags (spec S7); any nonzero flag means "malformed"
+// device status flags (spec S7); any nonzero flag other than kErrWait means
+// "malformed"; kErrWait: a bounded in-kernel wait ran out
 enum : uint32_t {
     kErrReserved = 1u << 0,
     kErrForm = 1u << 1,
@@ -34,6 +35,7 @@ enum : uint32_t {
     kErrPad = 1u << 7,
     kErrOffsets = 1u << 8,
     kErrValue = 1u << 9,
+    kErrWait = 1u << 31,
 };
 
 struct DevStatus {
@@ -116,16 +118,18 @@ cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const
 // decode_reduce reads count[0] heavy entries from list[0..) and count[1]
 // light entries from list[P - count[1], P).
 // plan: builds the signed pixel list, heavy class from the front (count[0]),
-// light class from the back (count[1]), and initialises the output rows:
-// mode 0 = full query (out = 0), 1 = delta (out = baseline image)
+// light class from the back (count[1]), clears count_next (the pair the next
+// query uses) and initialises the rows: mode 0 = full query (out = keep = 0),
+// 1 = delta (out = keep, the stride's kept image)
 cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t *pclass,
                         uint8_t *base_mask, int P, int mode, uint32_t *list, uint32_t *count,
-                        void *out, const void *base_img, long long n_elems, int out_bytes,
+                        uint32_t *count_next, void *out, void *keep, long long n_elems, int out_bytes,
                         cudaStream_t st);
+// keep (may be null): a second image that receives the same additions as out
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count,
                                  int stride, long long rows, void *out, int out_bytes,
-                                 DevStatus *status, int n_sm, cudaStream_t st, bool delta = false);
-cudaError_t launch_copy(void *dst, const void *src, size_t bytes, cudaStream_t st);
+                                 DevStatus *status, int n_sm, cudaStream_t st, bool delta = false,
+                                 void *keep = nullptr);
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out,
                                  DevStatus *status, cudaStream_t st);
 
