@@ -64,7 +64,7 @@ struct qem_resident {
     std::vector<Arena> arenas;
 
     uint32_t *d_dec = nullptr, *d_enc_sym = nullptr, *d_cost = nullptr, *d_amax = nullptr;
-    uint16_t *d_skip = nullptr;
+    uint32_t *d_runs = nullptr;
     uint32_t skip_models = 0;
     uint16_t *d_enc_slot = nullptr;
 
@@ -90,7 +90,7 @@ struct qem_resident {
     std::vector<ProfEvent> events;
     qem_profile_t prof_acc{};
 
-    Tables tables() const { return Tables{d_dec, d_enc_sym, d_enc_slot, d_cost, d_amax, d_skip, skip_models}; }
+    Tables tables() const { return Tables{d_dec, d_enc_sym, d_enc_slot, d_cost, d_amax, d_runs, skip_models}; }
     View view() const { return View{d_groups, d_blk_ptr, d_blk_len, d_valid, P, G, w, B}; }
 };
 
@@ -187,7 +187,7 @@ void release(qem_resident *r)
     cudaFree(r->d_enc_slot);
     cudaFree(r->d_cost);
     cudaFree(r->d_amax);
-    cudaFree(r->d_skip);
+    cudaFree(r->d_runs);
     cudaFree(r->d_desc);
     cudaFree(r->d_slots);
     cudaFree(r->d_stats);
@@ -259,7 +259,7 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
         (rc = dalloc(&r->d_blk_ptr, size_t(r->B) * 8)) || (rc = dalloc(&r->d_blk_len, size_t(r->B) * 4)) ||
         (rc = dalloc(&r->d_dec, sizeof(T.dec))) || (rc = dalloc(&r->d_enc_sym, sizeof(T.enc_sym))) ||
         (rc = dalloc(&r->d_enc_slot, sizeof(T.enc_slot))) || (rc = dalloc(&r->d_cost, sizeof(T.cost))) ||
-        (rc = dalloc(&r->d_amax, kModels * 4)) || (rc = dalloc(&r->d_skip, sizeof(T.skip))) || (rc = dalloc(&r->d_stats, (5 + kModels) * 8)) ||
+        (rc = dalloc(&r->d_amax, kModels * 4)) || (rc = dalloc(&r->d_runs, sizeof(T.runs))) || (rc = dalloc(&r->d_stats, (5 + kModels) * 8)) ||
         (rc = dalloc(&r->d_list, size_t(r->P) * 4)) || (rc = dalloc(&r->d_count, 16)) ||
         (rc = dalloc(&r->d_status, sizeof(DevStatus))))
         return fail(rc);
@@ -282,7 +282,7 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
     up(r->d_enc_slot, T.enc_slot, sizeof(T.enc_slot));
     up(r->d_cost, T.cost, sizeof(T.cost));
     up(r->d_amax, amax, sizeof(amax));
-    up(r->d_skip, T.skip, sizeof(T.skip));
+    up(r->d_runs, T.runs, sizeof(T.runs));
     r->skip_models = T.skip_models;
     if (e == cudaSuccess)
         e = cudaMemsetAsync(r->d_pclass, 0, hv.size(), st);

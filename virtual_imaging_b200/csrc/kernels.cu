@@ -993,7 +993,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
 // shared accumulator; the CTA then adds its rows to the output with one
 // global atomic per nonzero scan sum.
 template <int W, bool DELTA>
-__device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint16_t *skip,
+__device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint32_t *dec_g,
                                             uint32_t skip_models, const uint32_t *list, uint32_t n,
                                             uint32_t n_l, int tile,
                                             long long b, uint32_t *acc, uint32_t *stage, uint32_t *cnt,
@@ -1046,10 +1046,14 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
         atomicAdd(cnt + 1, nact);
     }
 
-    const uint32_t *dec = s_dec + S.model * kStates;
     // low-dose paired streams (models dominated by the (0,0) symbol) are decoded
-    // by runs after the per-scan loop instead of inside it
-    const bool runs = S.form == kPaired && S.shift == 0 && S.base == 0u && ((skip_models >> S.model) & 1u);
+    // by runs after the per-scan loop instead of inside it.  Those models'
+    // shared-memory slices hold their run tables; the rare stream of such a
+    // model that also has a base or raw bits reads its decode table from
+    // global memory (cached) instead.
+    const bool run_model = (skip_models >> S.model) & 1u;
+    const bool runs = S.form == kPaired && S.shift == 0 && S.base == 0u && run_model;
+    const uint32_t *dec = (run_model ? dec_g : s_dec) + S.model * kStates;
     const bool dense_lane = (S.form == kPaired && !runs) || S.form == kLiteral || S.form == kConstant;
     const bool fast = S.form == kPaired && !runs && S.shift == 0 && S.base == 0u;
     uint32_t over = 0;
@@ -1142,33 +1146,29 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     }
 
     if (runs) {
-        // Runs of zero-bit (0,0) steps are jumped with one table read; every
-        // other step is an ordinary tANS step whose nonzero counts are added
-        // to their scans.  A run that would pass pair 255 cannot end in the
+        // One event per iteration, one shared-memory read: jump the run of
+        // zero-bit (0,0) steps from the current state (possibly empty), then
+        // take the ordinary step at the slot reached, adding its nonzero
+        // counts to their scans.  A run that passes pair 255 cannot end in the
         // final state 1024 (that state reads bits), so it marks the stream
-        // malformed.  Each iteration advances j, so the loop ends.
-        const uint16_t *sk = skip + S.model * kStates;
+        // malformed; a run that ends exactly at pair 256 leaves the stream in
+        // the slot it reached, which the end check then requires to be 0.
+        // Each iteration advances j, so the loop ends.
+        const uint32_t *rt = s_dec + S.model * kStates;
         int j = 0;
         bool bad = false;
         while (j < kPairs) {
-            // a maximal run ends on a slot that reads bits or carries another
-            // symbol, so every iteration is: jump the run (if any), then one step
-            const uint32_t r = sk[S.x];
-            const int run = static_cast<int>(r >> 10);
-            if (run) {
-                j += run;
-                S.x = r & 1023u;
-                if (j >= kPairs) {
-                    bad = j > kPairs;
-                    break;
-                }
-                if (run == 63)
-                    continue;      // a capped run may go on from the slot it reached
+            const uint32_t t = rt[S.x];
+            j += static_cast<int>((t >> 14) & 63u);
+            if (j >= kPairs) {
+                bad = j > kPairs;
+                S.x = (t >> 28) & 1u;
+                break;
             }
             if (S.bt.n < 10)
                 S.bt.refill();
-            const uint32_t ent = tans_step(S, dec);
-            const uint32_t a = (ent >> 16) & 0xFFu, c = ent >> 24;
+            S.x = (t & 1023u) | S.bt.get(static_cast<int>((t >> 10) & 15u));
+            const uint32_t a = (t >> 20) & 15u, c = (t >> 24) & 15u;
             if (a)
                 atomicAdd(acc + 2 * j, neg ? 0u - a : a);
             if (c)
@@ -1220,7 +1220,7 @@ constexpr int kMaxSlots = 8;    // block rows one CTA range may touch (shared ac
 
 template <int W, int THREADS, bool DELTA>
 __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint32_t *__restrict__ dec_g,
-                                                             const uint16_t *__restrict__ skip_g,
+                                                             const uint32_t *__restrict__ runs_g,
                                                              uint32_t skip_models, int skip_count,
                                                              const uint32_t *__restrict__ list,
                                                              const uint32_t *__restrict__ count, int stride,
@@ -1229,17 +1229,18 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
                                                              DevStatus *__restrict__ st)
 {
     constexpr int MAXW = THREADS / 32;
-    // shared memory: decode tables of the 32 models | run tables of the first
-    // skip_count models | kMaxSlots per-row scan accumulators
+    // shared memory: one 4 KB table per model (the run tables of the first
+    // skip_count models, the decode tables of the others) | per-warp staging |
+    // kMaxSlots per-row scan accumulators
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *s_dec = smem;
-    uint16_t *s_skip = reinterpret_cast<uint16_t *>(smem + kModels * kStates);
-    uint32_t *s_stage = smem + kModels * kStates + skip_count * kStates / 2;   // 16 words per warp
+    uint32_t *s_stage = smem + kModels * kStates;   // 16 words per warp
     uint32_t *s_acc = s_stage + MAXW * 16;
     __shared__ __align__(8) uint64_t s_bar;
     if (threadIdx.x == 0)
-        tables_start(&s_bar, s_dec, dec_g, kModels * kStates * 4u, s_skip, skip_g,
-                     static_cast<uint32_t>(skip_count) * kStates * 2u);
+        tables_start(&s_bar, s_dec + skip_count * kStates, dec_g + skip_count * kStates,
+                     static_cast<uint32_t>(kModels - skip_count) * kStates * 4u, s_dec, runs_g,
+                     static_cast<uint32_t>(skip_count) * kStates * 4u);
     bool ready = false;
     // per-CTA counters (rows, streams), added to the status once at the end
     __shared__ uint32_t s_cnt[2];
@@ -1270,7 +1271,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
         if (warp < WARPS && task < total) {
             const long long row = task / tiles;
             const int tile = static_cast<int>(task - row * tiles);
-            decode_task<W, DELTA>(v, s_dec, s_skip, skip_models, list, n, n_l, tile, row * stride,
+            decode_task<W, DELTA>(v, s_dec, dec_g, skip_models, list, n, n_l, tile, row * stride,
                                   s_acc + (row - row0) * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready,
                                   lane, st);
         }
@@ -1505,7 +1506,7 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
 {
     // the run-decoded models are a prefix 0..k-1 (their (0,0) share falls as lambda grows)
     const int skip_count = __builtin_popcount(tb.skip_models);
-    const size_t smem = kTableBytes + static_cast<size_t>(skip_count) * kStates * sizeof(uint16_t) +
+    const size_t smem = kTableBytes +
                         static_cast<size_t>(TH / 32) * 16 * sizeof(uint32_t) +
                         static_cast<size_t>(kMaxSlots) * kScans * sizeof(uint32_t);
     static size_t attr = 0;
@@ -1516,7 +1517,7 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
             return e;
         attr = smem;
     }
-    k_decode_reduce<W, TH, DELTA><<<n_sm, TH, smem, st>>>(v, tb.dec, tb.skip, tb.skip_models, skip_count, list,
+    k_decode_reduce<W, TH, DELTA><<<n_sm, TH, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, list,
                                                           count, stride, rows, out, keep, out_bytes, status);
     return cudaGetLastError();
 }

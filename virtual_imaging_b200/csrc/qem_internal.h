@@ -19,6 +19,7 @@ constexpr int kModels = 32;        // Poisson pair models (page: 32)
 constexpr int kGroupWords = 17;    // 1 x u32 base + 32 x u16 relative ends (spec S1)
 constexpr int kSlotWords = 84;     // per-stream tANS scratch: >= ceil((10 + 256*10)/32) + 1 words, 16-byte multiple
 constexpr int kArenaPad = 64;      // zero bytes after the last block of an arena
+constexpr int kRunModels = 8;      // models that may be decoded by runs (their tables replace the decode tables in shared memory)
 
 enum Form : int { kEmpty = 0, kConstant = 1, kSparse = 2, kPaired = 3, kLiteral = 4 };
 
@@ -58,8 +59,8 @@ struct Tables {
     const uint16_t *enc_slot;
     const uint32_t *cost;
     const uint32_t *amax;
-    const uint16_t *skip;     // [m][slot]: run of zero-bit (0,0) steps from slot (bits 10-15, <= 63), slot after it (bits 0-9)
-    uint32_t skip_models;     // bit m set: model m's streams are decoded by runs
+    const uint32_t *runs;     // [m < kRunModels][slot]: one run event (see HostTables::runs)
+    uint32_t skip_models;     // bit m set: model m's streams are decoded by runs (a prefix of the models)
 };
 
 struct HostTables {
@@ -69,7 +70,13 @@ struct HostTables {
     uint32_t dec[kModels][kStates];
     uint32_t enc_sym[kModels][256];
     uint16_t enc_slot[kModels][kStates];
-    uint16_t skip[kModels][kStates];
+    // runs[m][slot], for the low-dose models m < kRunModels: from state slot,
+    // r = min(63, length of the chain of zero-bit (0,0) steps starting there)
+    // steps are jumped, landing on slot e; then e's ordinary decode step
+    // follows.  Bits 0-9 newbase(e), 10-13 nb(e), 14-19 r, 20-23 and 24-27 the
+    // two counts of e's symbol, 28: e != 0 (a stream may end on e only if e is
+    // state 1024, slot 0).
+    uint32_t runs[kRunModels][kStates];
     uint32_t skip_models;
 };
 

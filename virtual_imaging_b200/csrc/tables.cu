@@ -145,17 +145,24 @@ void make_runs(int m, HostTables &T)
             run[slot] = 1 + run[nx];
         }
     }
+    if (m >= kRunModels)
+        return;
+    bool small = true;      // every count of the model's symbols fits 4 bits
     for (int slot = 0; slot < kStates; ++slot) {
         const int r = run[slot] < 63 ? run[slot] : 63;
         int at = slot;
         for (int k = 0; k < r; ++k)
             at = next[at];
-        T.skip[m][slot] = r ? static_cast<uint16_t>((r << 10) | at) : static_cast<uint16_t>(0);
+        const uint32_t e = T.dec[m][at];
+        const uint32_t a = (e >> 16) & 0xFFu, c = e >> 24;
+        small = small && a < 16u && c < 16u;
+        T.runs[m][slot] = (e & 1023u) | (((e >> 10) & 15u) << 10) | (static_cast<uint32_t>(r) << 14) |
+                          ((a & 15u) << 20) | ((c & 15u) << 24) | (at != 0 ? 1u << 28 : 0u);
     }
     // decode by runs only where (0,0) holds at least 7/8 of the states (lambda
-    // up to ~0.04 here), a prefix of at most 8 models whose run tables live in
-    // shared memory; there a stream needs ~30-100 events instead of 256 steps
-    if (T.freq[m][0] >= 896 && m < 8 && (m == 0 || ((T.skip_models >> (m - 1)) & 1u)))
+    // up to ~0.04 here), a prefix of the first kRunModels models; there a
+    // stream needs ~15-40 events instead of 256 steps
+    if (small && T.freq[m][0] >= 896 && (m == 0 || ((T.skip_models >> (m - 1)) & 1u)))
         T.skip_models |= 1u << m;
 }
 
