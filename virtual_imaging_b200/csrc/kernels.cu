@@ -28,13 +28,12 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void report(DevStatus *st, uint32_t flag, long long b, int p)
+// Malformed-stream report (spec S7): a query only needs to know that some
+// stream failed, so a flag is all that is kept (recording where would keep the
+// block and pixel live through every decode loop).
+__device__ __forceinline__ void report(DevStatus *st, uint32_t flag)
 {
     atomicOr(&st->flags, flag);
-    if (atomicCAS(&st->have_first, 0u, 1u) == 0u) {
-        st->first_block = static_cast<uint32_t>(b);
-        st->first_pixel = static_cast<uint32_t>(p);
-    }
 }
 
 // Shared-memory tables arrive by the bulk-copy engine: one thread starts the
@@ -176,7 +175,7 @@ __device__ __forceinline__ bool locate(const View &v, long long b, int p, const 
     }
     const uint32_t blen = __ldg(v.blk_len + b);
     if (e1 < e0 || static_cast<uint64_t>(base) + e1 > blen) {
-        report(st, kErrOffsets, b, p);
+        report(st, kErrOffsets);
         return false;
     }
     s = reinterpret_cast<const uint8_t *>(__ldg(v.blk_ptr + b)) + base + e0;
@@ -197,7 +196,7 @@ __device__ __forceinline__ void prefetch_stream(const uint8_t *s, uint32_t len)
 }
 
 // Parse the header and set the readers up; false (after reporting) if malformed.
-__device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
+__device__ bool open_stream(Stream &S, int w, DevStatus *st)
 {
     if (S.len == 0) {
         S.form = kEmpty;
@@ -205,12 +204,12 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
     }
     prefetch_stream(S.s, S.len);
     if (S.len < 2) {
-        report(st, kErrLength, b, p);
+        report(st, kErrLength);
         return false;
     }
     const uint32_t hdr = static_cast<uint32_t>(__ldg(S.s)) | (static_cast<uint32_t>(__ldg(S.s + 1)) << 8);
     if (hdr >> 13) {
-        report(st, kErrReserved, b, p);
+        report(st, kErrReserved);
         return false;
     }
     S.form = static_cast<int>(hdr & 7);
@@ -218,29 +217,29 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
     S.shift = static_cast<int>((hdr >> 8) & 15);
     const int has_base = static_cast<int>((hdr >> 12) & 1);
     if (S.form < kConstant || S.form > kLiteral) {
-        report(st, kErrForm, b, p);
+        report(st, kErrForm);
         return false;
     }
     if (S.form != kPaired && (S.model | S.shift | has_base)) {
-        report(st, kErrFields, b, p);
+        report(st, kErrFields);
         return false;
     }
     const uint8_t *end = S.s + S.len;
     if (S.form == kConstant) {
         if (S.len != static_cast<uint32_t>(2 + w)) {
-            report(st, kErrLength, b, p);
+            report(st, kErrLength);
             return false;
         }
         S.c = load_native(S.s + 2, w);
         if (S.c == 0) {
-            report(st, kErrConstant, b, p);
+            report(st, kErrConstant);
             return false;
         }
         return true;
     }
     if (S.form == kLiteral) {
         if (S.len != static_cast<uint32_t>(2 + 512 * w)) {
-            report(st, kErrLength, b, p);
+            report(st, kErrLength);
             return false;
         }
         S.bt.init(S.s + 2, end);
@@ -248,13 +247,13 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
     }
     if (S.form == kSparse) {
         if (S.len < 3) {
-            report(st, kErrLength, b, p);
+            report(st, kErrLength);
             return false;
         }
         S.c = static_cast<uint32_t>(__ldg(S.s + 2)) + 1u;
         const uint32_t pbytes = (9u * S.c + 7u) / 8u;
         if (S.len != 3u + pbytes + S.c * static_cast<uint32_t>(w)) {
-            report(st, kErrLength, b, p);
+            report(st, kErrLength);
             return false;
         }
         S.bt.init(S.s + 3, end);
@@ -263,14 +262,14 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
     }
     // paired
     if (S.shift > 8 * w - 4) {
-        report(st, kErrFields, b, p);
+        report(st, kErrFields);
         return false;
     }
     uint32_t off = 2;
     S.base = 0;
     if (has_base) {
         if (S.len < off + static_cast<uint32_t>(w)) {
-            report(st, kErrLength, b, p);
+            report(st, kErrLength);
             return false;
         }
         S.base = load_native(S.s + off, w);
@@ -279,7 +278,7 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
     const uint32_t raw_off = off;
     off += 64u * static_cast<uint32_t>(S.shift);
     if (S.len < off + 2u) {
-        report(st, kErrLength, b, p);
+        report(st, kErrLength);
         return false;
     }
     S.tans_len = S.len - off;
@@ -293,15 +292,15 @@ __device__ bool open_stream(Stream &S, int w, long long b, int p, DevStatus *st)
 
 // End-of-stream checks of a paired stream (S5/S7): final state 1024, section
 // length exactly ceil(T/8), zero pad bits.
-__device__ bool close_paired(Stream &S, long long b, int p, DevStatus *st)
+__device__ bool close_paired(Stream &S, DevStatus *st)
 {
     if (S.x != 0) {
-        report(st, kErrState, b, p);
+        report(st, kErrState);
         return false;
     }
     const long long T = S.bt.consumed();
     if ((T + 7) / 8 != static_cast<long long>(S.tans_len)) {
-        report(st, kErrLength, b, p);
+        report(st, kErrLength);
         return false;
     }
     const int pad = static_cast<int>(8ll * S.tans_len - T);
@@ -309,7 +308,7 @@ __device__ bool close_paired(Stream &S, long long b, int p, DevStatus *st)
         if (S.bt.n < pad)
             S.bt.refill();
         if (S.bt.get(pad) != 0u) {
-            report(st, kErrPad, b, p);
+            report(st, kErrPad);
             return false;
         }
     }
@@ -1028,7 +1027,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     if (ok)
         ok = locate(v, b, p, S.s, S.len, st);
     if (ok)
-        ok = open_stream(S, W, b, p, st);
+        ok = open_stream(S, W, st);
     if (!ok)
         S.form = kEmpty;
     if (!ready) {
@@ -1176,14 +1175,14 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
             ++j;
         }
         if (bad)
-            report(st, kErrState, b, p);
+            report(st, kErrState);
         else
-            close_paired(S, b, p, st);
+            close_paired(S, st);
     } else if (S.form == kPaired) {
         if (over > (W == 1 ? 0xFFu : 0xFFFFu)) {
-            report(st, kErrValue, b, p);
+            report(st, kErrValue);
         }
-        close_paired(S, b, p, st);
+        close_paired(S, st);
     } else if (S.form == kSparse) {
         // sparse: scatter the nonzeros (positions strictly ascending, values nonzero)
         int prev = -1;
@@ -1203,14 +1202,14 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
             atomicAdd(acc + pos, neg ? 0u - val : val);
         }
         if (bad) {
-            report(st, kErrSparse, b, p);
+            report(st, kErrSparse);
         } else {
             const int pad = static_cast<int>(((9u * S.c + 7u) / 8u) * 8u - 9u * S.c);
             if (pad) {
                 if (S.bt.n < pad)
                     S.bt.refill();
                 if (S.bt.get(pad) != 0u)
-                    report(st, kErrPad, b, p);
+                    report(st, kErrPad);
             }
         }
     }
@@ -1343,7 +1342,7 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
         if (ok)
             ok = locate(v, b, p, S.s, S.len, st);
         if (ok)
-            ok = open_stream(S, W, b, p, st);
+            ok = open_stream(S, W, st);
         if (!ok)
             S.form = kEmpty;
         if (S.form == kPaired) {
@@ -1357,8 +1356,8 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
                     dst[(seg * 32 + i) * P] = static_cast<T>(vv[i]);
             }
             if (over > (W == 1 ? 0xFFu : 0xFFFFu))
-                report(st, kErrValue, b, p);
-            close_paired(S, b, p, st);
+                report(st, kErrValue);
+            close_paired(S, st);
         } else if (S.form == kLiteral) {
             for (int i = 0; i < kScans; ++i) {
                 if (S.bt.n < 16)
@@ -1387,14 +1386,14 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
             for (int i = prev + 1; i < kScans; ++i)
                 dst[i * P] = 0;
             if (bad) {
-                report(st, kErrSparse, b, p);
+                report(st, kErrSparse);
             } else {
                 const int pad = static_cast<int>(((9u * S.c + 7u) / 8u) * 8u - 9u * S.c);
                 if (pad) {
                     if (S.bt.n < pad)
                         S.bt.refill();
                     if (S.bt.get(pad) != 0u)
-                        report(st, kErrPad, b, p);
+                        report(st, kErrPad);
                 }
             }
         } else {

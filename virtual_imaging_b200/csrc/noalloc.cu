@@ -63,9 +63,6 @@ __global__ void __launch_bounds__(kPlanThreads) k_noalloc_plan(const uint8_t *__
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
         if (threadIdx.x == 0) {
             s->status.flags = 0u;
-            s->status.first_block = 0u;
-            s->status.first_pixel = 0u;
-            s->status.have_first = 0u;
             s->status.rows = 0ull;
             s->status.streams = 0ull;
         }

@@ -41,9 +41,7 @@ enum : uint32_t {
 
 struct DevStatus {
     uint32_t flags;
-    uint32_t first_block;
-    uint32_t first_pixel;
-    uint32_t have_first;
+    uint32_t reserved[3];
     unsigned long long rows;      // touched block rows decoded by masked sums
     unsigned long long streams;   // streams decoded by masked sums
 };
