@@ -1250,49 +1250,114 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     const uint32_t n_l = __ldg(count + 1);    // light entries, list[P - n_l, P)
     const long long tiles = ((n + 31u) >> 5) + ((n_l + 31u) >> 5);
     const long long total = rows * tiles;
-    // tasks per CTA range: up to one per warp, fewer when that spreads the work
-    // over more SMs, and few enough that a range touches at most kMaxSlots rows
-    const long long per = (total + gridDim.x - 1) / gridDim.x;
-    long long cap = (kMaxSlots - 1) * tiles + 1;
-    cap = cap < MAXW ? cap : MAXW;
-    const int WARPS = static_cast<int>(per < 1 ? 1 : (per > cap ? cap : per));
-    const long long ranges = (total + WARPS - 1) / WARPS;
+    // Each CTA owns one contiguous share [T0, T1) of the tasks (row-major:
+    // row, then tile); its warps take the next task from a shared counter as
+    // they finish, with no barrier between tasks.  Scan sums of a row gather
+    // in one of kMaxSlots shared slots; the warp that completes a row's last
+    // task in this share adds the slot to the output and frees it for the
+    // row kMaxSlots later.  Slots are 32-bit, so a row is cut into pieces of
+    // at most F tasks (F * 32 pixels of full-scale counts stay below 2^31 in
+    // magnitude); a piece ("vrow") is the unit that owns a slot.
+    constexpr long long kMaxCount = W == 1 ? 255 : 65535;
+    constexpr long long F = 0x7FFFFFFFll / (32 * kMaxCount);
+    const long long nch = (tiles + F - 1) / F;              // pieces per row
+    const long long T0 = total * blockIdx.x / gridDim.x, T1 = total * (blockIdx.x + 1) / gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (long long r = blockIdx.x; r < ranges; r += gridDim.x) {
-        const long long t0 = r * WARPS;
-        const long long row0 = t0 / tiles;
-        const long long tl = min(total - 1, t0 + WARPS - 1);
-        const int nslot = static_cast<int>(tl / tiles - row0 + 1);
-        for (int i = threadIdx.x; i < nslot * kScans; i += THREADS)
-            s_acc[i] = 0u;
-        __syncthreads();
-        const long long task = t0 + warp;
-        if (warp < WARPS && task < total) {
-            const long long row = task / tiles;
-            const int tile = static_cast<int>(task - row * tiles);
-            decode_task<W, DELTA>(v, s_dec, dec_g, skip_models, list, n, n_l, tile, row * stride,
-                                  s_acc + (row - row0) * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready,
-                                  lane, st);
-        }
-        __syncthreads();
-        for (int i = threadIdx.x; i < nslot * kScans; i += THREADS) {
-            const uint32_t val = s_acc[i];
-            if (val) {
-                const long long o = (row0 + i / kScans) * kScans + (i % kScans);
-                if (out_bytes == 4) {
-                    atomicAdd(reinterpret_cast<unsigned int *>(out) + o, val);
-                    if (keep)
-                        atomicAdd(reinterpret_cast<unsigned int *>(keep) + o, val);
-                } else {
-                    const unsigned long long wide =
-                        static_cast<unsigned long long>(static_cast<long long>(static_cast<int>(val)));
-                    atomicAdd(reinterpret_cast<unsigned long long *>(out) + o, wide);
-                    if (keep)
-                        atomicAdd(reinterpret_cast<unsigned long long *>(keep) + o, wide);
+    auto vrow_of = [&](long long t) {
+        const long long row = t / tiles;
+        return row * nch + (t - row * tiles) / F;
+    };
+    // tasks of piece vr inside [T0, T1)
+    auto piece_tasks = [&](long long vr) {
+        const long long row = vr / nch, c = vr - row * nch;
+        const long long a = row * tiles + c * F, b = row * tiles + min((c + 1) * F, tiles);
+        return max(0ll, min(b, T1) - max(a, T0));
+    };
+    __shared__ unsigned long long s_next;
+    __shared__ long long s_owner[kMaxSlots];
+    __shared__ uint32_t s_left[kMaxSlots];
+    __shared__ int s_abort;                   // set once a wait ran out: the CTA stops taking tasks
+    for (int i = threadIdx.x; i < kMaxSlots * kScans; i += THREADS)
+        s_acc[i] = 0u;
+    if (threadIdx.x == 0) {
+        s_next = static_cast<unsigned long long>(T0);
+        s_abort = 0;
+    }
+    if (threadIdx.x < kMaxSlots && T1 > T0) {
+        const long long v0 = vrow_of(T0);
+        const long long vr = v0 + ((threadIdx.x - v0) & (kMaxSlots - 1));
+        s_owner[threadIdx.x] = vr;
+        s_left[threadIdx.x] = static_cast<uint32_t>(vr <= vrow_of(T1 - 1) ? piece_tasks(vr) : 0);
+    }
+    __syncthreads();
+    while (true) {
+        long long t = 0;
+        if (lane == 0)
+            t = *reinterpret_cast<volatile int *>(&s_abort) ? T1 : static_cast<long long>(atomicAdd(&s_next, 1ull));
+        t = __shfl_sync(kFull, t, 0);
+        if (t >= T1)
+            break;
+        const long long row = t / tiles;
+        const int tile = static_cast<int>(t - row * tiles);
+        const long long vr = row * nch + tile / F;
+        const int slot = static_cast<int>(vr & (kMaxSlots - 1));
+        // the slot may still hold the piece kMaxSlots earlier: wait (bounded)
+        // until its last warp has emptied it.  That piece's tasks were all
+        // taken before this one, so the wait ends.
+        bool ok = true;
+        if (lane == 0) {
+            uint32_t it = 0;
+            while (*reinterpret_cast<volatile long long *>(&s_owner[slot]) != vr) {
+                if (++it > kWaitLimit) {
+                    atomicOr(&st->flags, kErrWait);
+                    *reinterpret_cast<volatile int *>(&s_abort) = 1;
+                    ok = false;
+                    break;
                 }
+                __nanosleep(32);
             }
         }
-        __syncthreads();
+        ok = __shfl_sync(kFull, ok, 0);
+        if (ok)
+            decode_task<W, DELTA>(v, s_dec, dec_g, skip_models, list, n, n_l, tile, row * stride,
+                                  s_acc + slot * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready, lane, st);
+        // this warp's slot additions happen before its count
+        __threadfence_block();
+        __syncwarp();
+        uint32_t left = 0;
+        if (lane == 0)
+            left = atomicSub(&s_left[slot], 1u);
+        left = __shfl_sync(kFull, left, 0);
+        if (left == 1u) {
+            __threadfence_block();
+            uint32_t *acc = s_acc + slot * kScans;
+            for (int i = lane; i < kScans; i += 32) {
+                const uint32_t val = acc[i];
+                if (val) {
+                    acc[i] = 0u;
+                    const long long o = row * kScans + i;
+                    if (out_bytes == 4) {
+                        atomicAdd(reinterpret_cast<unsigned int *>(out) + o, val);
+                        if (keep)
+                            atomicAdd(reinterpret_cast<unsigned int *>(keep) + o, val);
+                    } else {
+                        const unsigned long long wide =
+                            static_cast<unsigned long long>(static_cast<long long>(static_cast<int>(val)));
+                        atomicAdd(reinterpret_cast<unsigned long long *>(out) + o, wide);
+                        if (keep)
+                            atomicAdd(reinterpret_cast<unsigned long long *>(keep) + o, wide);
+                    }
+                }
+            }
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) {
+                const long long nv = vr + kMaxSlots;
+                s_left[slot] = static_cast<uint32_t>(nv <= vrow_of(T1 - 1) ? piece_tasks(nv) : 0);
+                __threadfence_block();
+                *reinterpret_cast<volatile long long *>(&s_owner[slot]) = nv;
+            }
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
