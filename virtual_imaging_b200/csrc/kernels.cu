@@ -916,6 +916,9 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
                                                       uint32_t *__restrict__ count_next, uint4 *__restrict__ out,
                                                       uint4 *__restrict__ keep, long long n_vec)
 {
+    // the decode that follows may start its prologue (table copy) now; it
+    // waits for this grid's completion before it reads anything written here
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (blockIdx.x == 0 && threadIdx.x < 2)
         count_next[threadIdx.x] = 0u;
     if (static_cast<int>(blockIdx.x) < n_list_blocks) {
@@ -1246,6 +1249,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     if (threadIdx.x < 2)
         s_cnt[threadIdx.x] = 0u;
 
+    // launched as a programmatic dependent of the plan: everything above only
+    // touched shared memory and the constant tables; wait here until the plan
+    // grid has finished and its list, counts and rows are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t n = __ldg(count);          // heavy entries, list[0, n)
     const uint32_t n_l = __ldg(count + 1);    // light entries, list[P - n_l, P)
     const long long tiles = ((n + 31u) >> 5) + ((n_l + 31u) >> 5);
@@ -1581,9 +1588,20 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
             return e;
         attr = smem;
     }
-    k_decode_reduce<W, TH, DELTA><<<n_sm, TH, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, list,
-                                                          count, stride, rows, out, keep, out_bytes, status);
-    return cudaGetLastError();
+    // programmatic dependent launch: the CTAs may become resident and load their
+    // tables while the preceding kernel (the plan) is still running
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_sm);
+    cfg.blockDim = dim3(TH);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_decode_reduce<W, TH, DELTA>, v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                              list, count, stride, rows, out, keep, out_bytes, status);
 }
 
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride,
