@@ -75,26 +75,68 @@ def stream_lengths(res, w):
     return lens
 
 
-def algorithmic_bytes(lens, w, sched, out_bits):
-    """Per query: encoded bytes of the listed streams in the touched blocks + 2 B offset per stream +
-    4 B group base per touched group + the image written + the 4 B list entries."""
+def decompose(slots, roots, P, add, rem):
+    """The plan's split of a query over the index layout: (items, residual pixels).
+    add/rem: bool [P] pixels entering / leaving the image (a full query has no rem).
+    Items are (level, id): a leaf whose every pixel enters (or every pixel leaves), or a
+    root whose leaves all do so in the same direction."""
+    real = slots < P
+    px = np.where(real, slots, 0)
+    a = np.where(real, add[px], True).all(axis=1)
+    r = np.where(real, rem[px], True).all(axis=1) & rem.any()
+    state = np.where(a, 1, np.where(r, 2, 0))
+    items, covered = [], np.zeros(slots.shape[0], bool)
+    for i in range(len(roots) - 1):
+        s = state[roots[i]:roots[i + 1]]
+        if s[0] > 0 and (s == s[0]).all():
+            items.append((1, i))
+            covered[roots[i]:roots[i + 1]] = True
+        else:
+            for l in range(roots[i], roots[i + 1]):
+                if state[l] > 0:
+                    items.append((0, l))
+                    covered[l] = True
+    cov = np.zeros(P, bool)
+    cov[slots[covered][slots[covered] < P]] = True
+    resid = (add | rem) & ~cov
+    return items, resid
+
+
+def algorithmic_bytes(lens, w, sched, out_bits, idx=None):
+    """Per query: encoded bytes of the decoded streams in the touched blocks + 2 B offset per stream +
+    4 B group base per touched group + the image written + the 4 B list entries; with the index
+    (idx = (slots, roots, bytes [B][L+R])), the residual pixels' streams plus the stored sums of
+    the index items in the touched blocks and 4 B per item."""
     out = []
     prev = None
     for label, m, k, delta in sched:
         sel = m.astype(bool)
-        if delta and prev is not None:
-            lst = sel ^ prev
+        as_delta = delta and prev is not None        # a delta with no baseline runs as a full query
+        if as_delta:
+            add, rem = sel & ~prev, ~sel & prev
         else:
-            lst = sel
+            add, rem = sel, np.zeros_like(sel)
         prev = sel
-        pix = np.nonzero(lst)[0]
         rows = list(range(0, w.n_blocks, k))
+        items = []
+        resid = add | rem
+        if idx is not None and not as_delta:           # deltas take the per-pixel plan
+            slots, roots, gbytes = idx
+            items, resid = decompose(slots, roots, w.n_pixels, add, rem)
+        pix = np.nonzero(resid)[0]
         enc = int(lens[rows][:, pix].sum(dtype=np.int64))
         groups = len(np.unique(pix // 32)) * len(rows)
+        isum = 0
+        if items:
+            L = slots.shape[0]
+            gid = np.array([g if lvl == 0 else L + g for lvl, g in items])
+            isum = int(gbytes[rows][:, gid].sum(dtype=np.int64))
         img = len(rows) * 512 * out_bits // 8
-        raw = pix.size * 512 * len(rows) * (w.dtype_bits // 8)
-        out.append(dict(label=label, enc=enc, streams=pix.size * len(rows), bytes=enc + 2 * pix.size * len(rows)
-                        + 4 * groups + img + 4 * pix.size, raw=raw))
+        listed = np.count_nonzero(add | rem)
+        raw = listed * 512 * len(rows) * (w.dtype_bits // 8)
+        out.append(dict(label=label, enc=enc + isum, streams=pix.size * len(rows), items=len(items),
+                        bytes=enc + 2 * pix.size * len(rows) + 4 * groups + isum + 4 * len(items) + img + 4 * pix.size,
+                        raw=raw))
     return out
 
 
@@ -294,6 +336,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="c4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-index", action="store_true",
+                    help="query without the interaction index (every masked pixel decoded)")
     ap.add_argument("--profile", action="store_true", help="bounded case for ncu captures")
     ap.add_argument("--profile-encode", action="store_true", help="bounded encode case for ncu captures")
     args = ap.parse_args()
@@ -325,6 +369,19 @@ def main():
         return
     w = W.workload(args.config)
     res, buf, _ = build_resident(w, dev, torch, V)
+    # interaction index about the detector centre (the centre of the bright-field
+    # disk and of the annulus); built by decoding every stream once
+    index = None
+    if not args.no_index:
+        torch.cuda.synchronize()
+        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        i0.record()
+        res.build_index((w.det_rows // 2, w.det_cols // 2))
+        i1.record()
+        torch.cuda.synchronize()
+        ii = res.info()
+        index = {"s": i0.elapsed_time(i1) / 1e3, "bytes": ii["index_bytes"], "leaves": ii["index_leaves"],
+                 "roots": ii["index_roots"], "centre": [w.det_rows // 2, w.det_cols // 2]}
     # a second, warm encode of the same counts for the encode figure (chunked workloads keep the first)
     enc_s = None
     enc_prof = None
@@ -466,7 +523,13 @@ def main():
 
     # per-query breakdown (separate, untimed for `value`)
     lens = stream_lengths(res, w)
-    ab = algorithmic_bytes(lens, w, sched, out_bits)
+    idx = None
+    if index is not None:
+        slots, roots = res.index_layout()
+        codes = res.index_desc() >> 30
+        gbytes = np.where(codes > 0, 512 << np.maximum(codes.astype(np.int64) - 1, 0), 0)
+        idx = (slots, roots, gbytes)
+    ab = algorithmic_bytes(lens, w, sched, out_bits, idx)
     per_query = {}
     for (label, m, k, delta), md, a in zip(sched, masks, ab):
         q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -523,6 +586,7 @@ def main():
                    "kernel_gbs_raw": (w.raw_bytes / (sum(enc_prof.values()) / 1e3) / 1e9) if enc_prof else None,
                    "hbm_frac": ((w.raw_bytes + info["payload_bytes"] + info["group_bytes"]) / enc_s / 1e9 / hbm)
                    if enc_s else None},
+        "index": index,
         "decode_blocks": {"blocks": nd, "s": dec_s, "gcounts_per_s": nd * 512 * w.n_pixels / dec_s / 1e9,
                           "exact": ok_frames},
         "resident": {"payload_bytes": info["payload_bytes"], "forms": info["form_count"],

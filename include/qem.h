@@ -65,6 +65,9 @@ typedef struct {
     uint64_t form_count[5];         /* streams per form: empty, constant, sparse, paired, literal */
     uint64_t model_count[32];       /* paired streams per model                        */
     int32_t n_arenas;               /* payload allocations                             */
+    int32_t index_leaves;           /* interaction index: leaves (0 = no index)        */
+    int32_t index_roots;            /* interaction index: roots                        */
+    uint64_t index_bytes;           /* interaction index: stored sums                  */
 } qem_info_t;
 
 /* Per-kernel device time, gathered with CUDA events on the launching stream
@@ -151,6 +154,77 @@ int qem_masked_sum_delta(qem_resident *res, const uint8_t *d_new_mask, int32_t b
  * in the native dtype (aligned to it), invalid pixels 0.  Same wait rule as the queries. */
 int qem_decode_blocks(qem_resident *res, int64_t first_block, int64_t n_blocks, void *d_out,
                       int32_t wait, void *stream);
+
+/* Interaction index (page "Operation pipeline" step 3: exact per-scan sums of
+ * radial-angular pixel groups, 64-pixel leaves and 16-leaf roots; step 4: a
+ * mask, or its difference from the previous mask, is decomposed into index
+ * groups plus residual pixels).  Builds the index of a complete resident by
+ * decoding every stream once: the valid pixels are split into 16 angular
+ * sectors about (center_row, center_col) (detector pixel coordinates, may be
+ * fractional), sorted by distance inside each sector and cut into leaves of
+ * 64; 16 consecutive leaves of a sector form a root.  For every block and
+ * group the 512 sums are kept at 1, 2 or 4 bytes each (the smallest that
+ * holds the group's largest sum in that block; none when all are zero).
+ * Afterwards every full masked sum (any stride) takes whole groups from the
+ * index and decodes only the remaining pixels; a delta decodes its changed
+ * pixels (an edge that moves rarely fills a whole group); results are
+ * unchanged (exact).  Rebuilding replaces the index; it synchronises
+ * `stream` first.  Errors: QEM_ERR_ARG (null resident, centre not finite),
+ * QEM_ERR_STATE (resident not complete), QEM_ERR_MALFORMED (a stream failed
+ * its checks while summing; no index is kept), QEM_ERR_OOM, QEM_ERR_CUDA. */
+int qem_build_index(qem_resident *res, double center_row, double center_col, void *stream);
+
+/* Discard the interaction index (queries decode every masked pixel again).
+ * Synchronises `stream` first. */
+int qem_drop_index(qem_resident *res, void *stream);
+
+/* The index's polar layout, for inspection: *n_leaves and *n_roots (may be
+ * NULL); h_slots (host, may be NULL) receives 64 pixel indices per leaf, in
+ * leaf order, with n_pixels marking unused slots of a sector's last leaf;
+ * h_root_leaf0 (host, may be NULL) receives n_roots + 1 entries, root r
+ * holding leaves [h_root_leaf0[r], h_root_leaf0[r + 1]).  QEM_ERR_STATE when
+ * the resident has no index. */
+int qem_index_layout(const qem_resident *res, uint32_t *h_slots, int32_t *h_root_leaf0, int32_t *n_leaves,
+                     int32_t *n_roots);
+
+/* The validity map the resident was created with: h_valid (host, n_pixels
+ * bytes) receives 1 for valid and 0 for invalid pixels. */
+int qem_export_valid(const qem_resident *res, uint8_t *h_valid);
+
+/* Saved form (page "Contract": saved form; "Operation pipeline" step 5: the
+ * resident arrays are written once and reopened with no decode).  qem_save
+ * writes a complete resident to `path`: the magic "QGPUPAIR", a u32 header
+ * length, a JSON header (format "qem-pair-resident-v1", the ABI string, the
+ * geometry and each array's offset and length), then 4096-byte aligned arrays:
+ * the validity map, the group records, the u64 block payload offsets and the
+ * payload bytes.  The interaction index is not saved (qem_build_index
+ * rebuilds it).  Errors: QEM_ERR_ARG (null argument, file not writable),
+ * QEM_ERR_STATE (resident not complete), QEM_ERR_CUDA. */
+int qem_save(const qem_resident *res, const char *path, void *stream);
+
+/* Reopen a saved form as a new resident (*out; free with qem_free).  The
+ * magic, the format and the ABI string must match this library's
+ * ("reopen refuses another ABI"); sizes and offsets are checked.  The streams
+ * themselves are checked when queried, as for qem_import.  Errors:
+ * QEM_ERR_ARG (unreadable, truncated or foreign file), QEM_ERR_OOM,
+ * QEM_ERR_CUDA. */
+int qem_load(const char *path, void *stream, qem_resident **out);
+
+/* The index's storage descriptors, for inspection and byte accounting: h_desc
+ * (host) receives n_blocks x (n_leaves + n_roots) words, group g of block b at
+ * [b * (n_leaves + n_roots) + g] (roots after the leaves); bits 30-31 give the
+ * width of its 512 sums (0: all zero and not stored; 1, 2, 3: 1, 2, 4 bytes),
+ * bits 0-29 the byte offset in the block's index storage.  QEM_ERR_STATE when
+ * the resident has no index. */
+int qem_index_desc(const qem_resident *res, uint32_t *h_desc);
+
+/* Block decode plus amplitude (page "Operation pipeline" step 6: the feed's
+ * "counts plus float32 sqrt amplitude"): as qem_decode_blocks into d_counts,
+ * then d_amp (float32, same [n_blocks*512][pixels] shape, 4-byte aligned)
+ * receives sqrtf(count) of every decoded count (correctly rounded; invalid
+ * pixels 0).  Same wait rule and errors as qem_decode_blocks. */
+int qem_decode_blocks_amplitude(qem_resident *res, int64_t first_block, int64_t n_blocks, void *d_counts,
+                                float *d_amp, int32_t wait, void *stream);
 
 /* Wait (bounded, ~60 s) for all queued work on `stream` and report any
  * malformed stream found since the last qem_finish (page "Contract":

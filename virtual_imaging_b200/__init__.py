@@ -30,7 +30,9 @@ FORMS = ("empty", "constant", "sparse", "paired", "literal")
 EXPORTS = ("qem_abi", "qem_status_string", "qem_create", "qem_encode", "qem_encode_append", "qem_masked_sum",
            "qem_masked_sum_delta", "qem_decode_blocks", "qem_finish", "qem_info", "qem_query_counters",
            "qem_profile", "qem_profile_read", "qem_free", "qem_block_bytes", "qem_export_block", "qem_import",
-           "qem_model_tables", "qem_generate_counts", "qem_masked_sum_noalloc")
+           "qem_model_tables", "qem_generate_counts", "qem_masked_sum_noalloc", "qem_build_index",
+           "qem_drop_index", "qem_index_layout", "qem_index_desc", "qem_export_valid", "qem_save", "qem_load",
+           "qem_decode_blocks_amplitude")
 
 
 class QemError(RuntimeError):
@@ -54,7 +56,8 @@ class Info(ctypes.Structure):
                 ("n_blocks_encoded", ctypes.c_int64), ("payload_bytes", ctypes.c_uint64),
                 ("group_bytes", ctypes.c_uint64), ("device_bytes", ctypes.c_uint64),
                 ("form_count", ctypes.c_uint64 * 5), ("model_count", ctypes.c_uint64 * 32),
-                ("n_arenas", ctypes.c_int32)]
+                ("n_arenas", ctypes.c_int32), ("index_leaves", ctypes.c_int32), ("index_roots", ctypes.c_int32),
+                ("index_bytes", ctypes.c_uint64)]
 
 
 class Profile(ctypes.Structure):
@@ -96,6 +99,14 @@ def lib() -> ctypes.CDLL:
         "qem_model_tables": ([vp, vp, vp], ctypes.c_int),
         "qem_generate_counts": ([vp, i32, u64, i64, i64, i32, vp, vp, vp, vp], ctypes.c_int),
         "qem_masked_sum_noalloc": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
+        "qem_build_index": ([vp, ctypes.c_double, ctypes.c_double, vp], ctypes.c_int),
+        "qem_drop_index": ([vp, vp], ctypes.c_int),
+        "qem_index_layout": ([vp, vp, vp, ctypes.POINTER(i32), ctypes.POINTER(i32)], ctypes.c_int),
+        "qem_index_desc": ([vp, vp], ctypes.c_int),
+        "qem_export_valid": ([vp, vp], ctypes.c_int),
+        "qem_save": ([vp, ctypes.c_char_p, vp], ctypes.c_int),
+        "qem_load": ([ctypes.c_char_p, vp, pp], ctypes.c_int),
+        "qem_decode_blocks_amplitude": ([vp, i64, i64, vp, vp, i32, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -248,6 +259,65 @@ class Resident:
         _check(lib().qem_decode_blocks(self._h, first, n, _dev_ptr(out), 1 if wait else 0, _stream(stream)),
                "qem_decode_blocks")
         return out
+
+    # ---- interaction index ----------------------------------------------------
+    def build_index(self, center=None, stream=None):
+        """Build the interaction index about `center` (detector row, col; default the detector centre)."""
+        if center is None:
+            i = self.info()
+            center = ((i["det_rows"] - 1) / 2.0, (i["det_cols"] - 1) / 2.0)
+        _check(lib().qem_build_index(self._h, float(center[0]), float(center[1]), _stream(stream)),
+               "qem_build_index")
+
+    def drop_index(self, stream=None):
+        _check(lib().qem_drop_index(self._h, _stream(stream)), "qem_drop_index")
+
+    def index_layout(self):
+        """(slots int64 [leaves][64] with n_pixels for unused slots, root_leaf0 int64 [roots + 1])."""
+        nl, nr = ctypes.c_int32(0), ctypes.c_int32(0)
+        _check(lib().qem_index_layout(self._h, None, None, ctypes.byref(nl), ctypes.byref(nr)), "qem_index_layout")
+        slots = np.zeros((nl.value, 64), np.uint32)
+        roots = np.zeros(nr.value + 1, np.int32)
+        _check(lib().qem_index_layout(self._h, slots.ctypes.data, roots.ctypes.data, None, None), "qem_index_layout")
+        return slots.astype(np.int64), roots.astype(np.int64)
+
+    # ---- saved form -------------------------------------------------------------
+    def save(self, path: str, stream=None):
+        """Write the resident's saved form (QGPUPAIR file) to `path`."""
+        _check(lib().qem_save(self._h, os.fsencode(path), _stream(stream)), "qem_save")
+
+    @classmethod
+    def load(cls, path: str, stream=None):
+        """Reopen a saved form written by save()."""
+        h = ctypes.c_void_p()
+        _check(lib().qem_load(os.fsencode(path), _stream(stream), ctypes.byref(h)), "qem_load")
+        return cls(h)
+
+    def valid(self) -> np.ndarray:
+        i = self.info()
+        v = np.zeros(i["n_pixels"], np.uint8)
+        _check(lib().qem_export_valid(self._h, v.ctypes.data), "qem_export_valid")
+        return v
+
+    def index_desc(self):
+        """uint32 [n_blocks][leaves + roots] storage descriptors (width code in bits 30-31)."""
+        i = self.info()
+        d = np.zeros((i["n_blocks"], i["index_leaves"] + i["index_roots"]), np.uint32)
+        _check(lib().qem_index_desc(self._h, d.ctypes.data), "qem_index_desc")
+        return d
+
+    def decode_blocks_amplitude(self, first: int, n: int, counts: torch.Tensor | None = None,
+                                amp: torch.Tensor | None = None, wait: bool = True, stream=None):
+        """(counts [n*512][P] native, amplitude float32 sqrt(counts) of the same shape)."""
+        _, n_pixels, bits, _ = self._static()
+        dev = torch.device("cuda", torch.cuda.current_device())
+        if counts is None:
+            counts = torch.empty((n * 512, n_pixels), dtype=_count_dtype(bits), device=dev)
+        if amp is None:
+            amp = torch.empty((n * 512, n_pixels), dtype=torch.float32, device=dev)
+        _check(lib().qem_decode_blocks_amplitude(self._h, first, n, _dev_ptr(counts), _dev_ptr(amp),
+                                                 1 if wait else 0, _stream(stream)), "qem_decode_blocks_amplitude")
+        return counts, amp
 
     def finish(self, stream=None):
         _check(lib().qem_finish(self._h, _stream(stream)), "qem_finish")

@@ -4,9 +4,12 @@
 // Page "Paired-count resident layout": "Operation pipeline" steps 1-6 and
 // "Contract" (virtual image dtype rule, malformed streams raise, queued
 // queries with a failed decode invalidating the incremental plan).
+#include <algorithm>
 #include <chrono>
+#include <cmath>
 #include <cstring>
 #include <map>
+#include <numeric>
 #include <thread>
 #include <vector>
 
@@ -77,8 +80,21 @@ struct qem_resident {
     size_t pinned_blocks = 0;
 
     uint32_t *d_list = nullptr;
-    uint32_t *d_count = nullptr;                // two (heavy, light) counter pairs, used in turn
-    int count_pair = 0;                         // the pair the next query fills
+    uint32_t *d_count = nullptr;                // two sets of (heavy, light, items, -) counters, used in turn
+    int count_pair = 0;                         // the set the next query fills
+    std::vector<uint8_t> h_valid;
+
+    // interaction index (page "Operation pipeline" step 3)
+    bool has_index = false;
+    int idx_L = 0, idx_R = 0;
+    double idx_center[2] = {0.0, 0.0};
+    uint32_t *d_idx_slots = nullptr;            // [64 L] pixel of each polar slot (P = padding)
+    int *d_idx_root_leaf0 = nullptr;            // [R + 1]
+    uint32_t *d_idx_desc = nullptr;             // [B][L + R]
+    unsigned long long *d_idx_base = nullptr;   // [B]
+    uint32_t *d_idx_items = nullptr;            // [L + R] items of the current query
+    std::vector<Arena> idx_arenas;
+    uint64_t idx_bytes = 0;
     DevStatus *d_status = nullptr;
     DevStatus *h_status = nullptr;              // pinned
     std::map<int, Baseline> baselines;
@@ -173,6 +189,13 @@ void release(qem_resident *r)
     }
     for (auto &a : r->arenas)
         cudaFree(a.p);
+    for (auto &a : r->idx_arenas)
+        cudaFree(a.p);
+    cudaFree(r->d_idx_slots);
+    cudaFree(r->d_idx_root_leaf0);
+    cudaFree(r->d_idx_desc);
+    cudaFree(r->d_idx_base);
+    cudaFree(r->d_idx_items);
     for (auto &kv : r->baselines) {
         cudaFree(kv.second.d_mask);
         cudaFree(kv.second.d_img);
@@ -252,6 +275,7 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
         x = x ? 1 : 0;
         r->n_valid += x;
     }
+    r->h_valid = hv;
     r->out_bits_auto = static_cast<uint64_t>(r->n_valid) * ((1ull << bits) - 1ull) > 0xFFFFFFFFull ? 64 : 32;
 
     const HostTables &T = host_tables();
@@ -260,10 +284,10 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
         (rc = dalloc(&r->d_dec, sizeof(T.dec))) || (rc = dalloc(&r->d_enc_sym, sizeof(T.enc_sym))) ||
         (rc = dalloc(&r->d_enc_slot, sizeof(T.enc_slot))) || (rc = dalloc(&r->d_cost, sizeof(T.cost))) ||
         (rc = dalloc(&r->d_amax, kModels * 4)) || (rc = dalloc(&r->d_runs, sizeof(T.runs))) || (rc = dalloc(&r->d_stats, (5 + kModels) * 8)) ||
-        (rc = dalloc(&r->d_list, size_t(r->P) * 4)) || (rc = dalloc(&r->d_count, 16)) ||
+        (rc = dalloc(&r->d_list, size_t(r->P) * 4)) || (rc = dalloc(&r->d_count, 32)) ||
         (rc = dalloc(&r->d_status, sizeof(DevStatus))))
         return fail(rc);
-    if (cudaMemset(r->d_count, 0, 16) != cudaSuccess)
+    if (cudaMemset(r->d_count, 0, 32) != cudaSuccess)
         return fail(QEM_ERR_CUDA);
     if (cudaMallocHost(&r->h_status, sizeof(DevStatus)) != cudaSuccess)
         return fail(QEM_ERR_OOM);
@@ -421,9 +445,17 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         if (bl.state == kValid && bl.out_bits == bits)
             mode = 1;
     }
-    uint32_t *count = r->d_count + 2 * r->count_pair;
-    uint32_t *count_next = r->d_count + 2 * (r->count_pair ^ 1);
+    uint32_t *count = r->d_count + 4 * r->count_pair;
+    uint32_t *count_next = r->d_count + 4 * (r->count_pair ^ 1);
+    // The index plan serves full queries; a delta lists its changed pixels one by
+    // one (a moving mask changes pixels along its edge, which rarely fill a whole
+    // group, and the per-pixel plan is the shorter launch).
+    const bool use_index = r->has_index && mode == 0;
     int rc = timed(r, QEM_K_PLAN, st, [&] {
+        if (use_index)
+            return launch_plan_index(d_mask, r->d_pclass, bl.d_mask, r->P, mode, r->d_idx_slots, r->d_idx_root_leaf0,
+                                     r->idx_R, r->d_list, r->d_idx_items, count, count_next, d_out, bl.d_img,
+                                     n_elems, bits / 8, st);
         return launch_plan(d_mask, r->d_valid, r->d_pclass, bl.d_mask, r->P, mode, r->d_list, count, count_next,
                            d_out, bl.d_img, n_elems, bits / 8, st);
     });
@@ -433,8 +465,11 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
     // the decode adds every term to d_out and to the stride's kept image, so
     // the kept image is this query's result without a copy
     rc = timed(r, QEM_K_DECODE_REDUCE, st, [&] {
+        const IndexView ix = use_index ? IndexView{r->d_idx_desc, r->d_idx_base, r->d_idx_items, r->idx_L,
+                                                      r->idx_L + r->idx_R}
+                                          : IndexView{nullptr, nullptr, nullptr, 0, 0};
         return launch_decode_reduce(r->view(), r->tables(), r->d_list, count, k, rows, d_out, bits / 8,
-                                    r->d_status, r->n_sm, st, mode == 1, bl.d_img);
+                                    r->d_status, r->n_sm, st, mode == 1, bl.d_img, ix);
     });
     if (rc)
         return rc;
@@ -453,6 +488,183 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         return report_errors(r, st);
     }
     return QEM_OK;
+}
+
+// Polar layout of the interaction index (page "Operation pipeline" step 3:
+// radial-angular pixel groups, 64-pixel leaves, 16-leaf roots).  Reading:
+// the valid pixels are split into 16 angular sectors around the centre
+// (boundaries every 22.5 degrees, so the row and column axes through the
+// centre are sector edges), ordered by distance inside each sector (then by
+// angle and index), and cut into leaves of 64 consecutive pixels; 16
+// consecutive leaves of one sector form a root.  A disk or annulus about the
+// centre then covers whole leaves and roots except along its two circles, and
+// a quadrant of one covers whole leaves except along its arc.
+struct PolarLayout {
+    std::vector<uint32_t> slots;     // [64 L], padding = P
+    std::vector<int> root_leaf0;     // [R + 1]
+    int L = 0, R = 0;
+};
+
+PolarLayout polar_layout(int det_rows, int det_cols, const std::vector<uint8_t> &valid, double cr, double cc)
+{
+    constexpr int kSectors = 16;
+    const double two_pi = 6.283185307179586;
+    struct Px {
+        int sector;
+        double d2, ang;
+        int p;
+    };
+    std::vector<std::vector<Px>> sec(kSectors);
+    for (int r = 0; r < det_rows; ++r)
+        for (int c = 0; c < det_cols; ++c) {
+            const int p = r * det_cols + c;
+            if (!valid[p])
+                continue;
+            const double dr = r - cr, dc = c - cc;
+            double a = std::atan2(dr, dc);          // (-pi, pi]
+            if (a < 0)
+                a += two_pi;                        // [0, 2 pi)
+            int s = static_cast<int>(a / (two_pi / kSectors));
+            s = s < 0 ? 0 : (s >= kSectors ? kSectors - 1 : s);
+            sec[s].push_back(Px{s, dr * dr + dc * dc, a, p});
+        }
+    PolarLayout out;
+    const uint32_t P = static_cast<uint32_t>(det_rows) * static_cast<uint32_t>(det_cols);
+    for (auto &v : sec) {
+        std::sort(v.begin(), v.end(), [](const Px &x, const Px &y) {
+            if (x.d2 != y.d2)
+                return x.d2 < y.d2;
+            if (x.ang != y.ang)
+                return x.ang < y.ang;
+            return x.p < y.p;
+        });
+        const int leaves = static_cast<int>((v.size() + 63) / 64);
+        for (int l = 0; l < leaves; ++l) {
+            if (l % 16 == 0)
+                out.root_leaf0.push_back(out.L);
+            for (int k = 0; k < 64; ++k) {
+                const size_t i = static_cast<size_t>(l) * 64 + k;
+                out.slots.push_back(i < v.size() ? static_cast<uint32_t>(v[i].p) : P);
+            }
+            ++out.L;
+        }
+    }
+    out.R = static_cast<int>(out.root_leaf0.size());
+    out.root_leaf0.push_back(out.L);
+    return out;
+}
+
+void drop_index(qem_resident *r)
+{
+    for (auto &a : r->idx_arenas)
+        cudaFree(a.p);
+    r->idx_arenas.clear();
+    cudaFree(r->d_idx_slots);
+    cudaFree(r->d_idx_root_leaf0);
+    cudaFree(r->d_idx_desc);
+    cudaFree(r->d_idx_base);
+    cudaFree(r->d_idx_items);
+    r->d_idx_slots = nullptr;
+    r->d_idx_root_leaf0 = nullptr;
+    r->d_idx_desc = nullptr;
+    r->d_idx_base = nullptr;
+    r->d_idx_items = nullptr;
+    r->has_index = false;
+    r->idx_L = r->idx_R = 0;
+    r->idx_bytes = 0;
+}
+
+// Reserve n bytes (512-aligned) of index storage; returns the device address.
+int place_index(qem_resident *r, uint64_t n, unsigned long long &ptr)
+{
+    const uint64_t need = (n + 511) & ~uint64_t(511);
+    if (r->idx_arenas.empty() || r->idx_arenas.back().used + need > r->idx_arenas.back().cap) {
+        Arena a;
+        a.cap = std::max<size_t>(need, size_t(256) << 20);
+        void *q = nullptr;
+        if (cudaMalloc(&q, a.cap) != cudaSuccess)
+            return QEM_ERR_OOM;
+        a.p = static_cast<uint8_t *>(q);
+        r->idx_arenas.push_back(a);
+    }
+    Arena &a = r->idx_arenas.back();
+    ptr = reinterpret_cast<unsigned long long>(a.p + a.used);
+    a.used += need;
+    r->idx_bytes += n;
+    return QEM_OK;
+}
+
+int build_index(qem_resident *r, double cr, double cc, cudaStream_t st)
+{
+    drop_index(r);
+    PolarLayout lay = polar_layout(r->det_rows, r->det_cols, r->h_valid, cr, cc);
+    r->idx_L = lay.L;
+    r->idx_R = lay.R;
+    r->idx_center[0] = cr;
+    r->idx_center[1] = cc;
+    const int L = lay.L, R = lay.R, G = L + R;
+    if (L == 0)
+        return QEM_OK;      // no valid pixels: nothing to index
+    int rc;
+    if ((rc = dalloc(&r->d_idx_slots, lay.slots.size() * 4)) ||
+        (rc = dalloc(&r->d_idx_root_leaf0, lay.root_leaf0.size() * 4)) ||
+        (rc = dalloc(&r->d_idx_desc, static_cast<size_t>(r->B) * G * 4)) ||
+        (rc = dalloc(&r->d_idx_base, static_cast<size_t>(r->B) * 8)) ||
+        (rc = dalloc(&r->d_idx_items, static_cast<size_t>(G) * 4)))
+        return rc;
+    QEM_CK(cudaMemcpyAsync(r->d_idx_slots, lay.slots.data(), lay.slots.size() * 4, cudaMemcpyHostToDevice, st));
+    QEM_CK(cudaMemcpyAsync(r->d_idx_root_leaf0, lay.root_leaf0.data(), lay.root_leaf0.size() * 4,
+                           cudaMemcpyHostToDevice, st));
+    // blocks per batch: leaf sums of about 64 MB
+    const size_t per_block = static_cast<size_t>(L) * kScans * 4;
+    int64_t nb = static_cast<int64_t>((size_t(64) << 20) / per_block);
+    nb = nb < 1 ? 1 : (nb > r->B ? r->B : nb);
+    nb = nb > 32768 ? 32768 : nb;           // grid y of the pack kernel
+    uint32_t *leafsum = nullptr;
+    unsigned long long *d_total = nullptr;
+    std::vector<unsigned long long> total(static_cast<size_t>(nb)), base(static_cast<size_t>(r->B));
+    auto cleanup = [&](int code) {
+        cudaFree(leafsum);
+        cudaFree(d_total);
+        if (code != QEM_OK)
+            drop_index(r);
+        return code;
+    };
+    if ((rc = dalloc(&leafsum, per_block * nb)) || (rc = dalloc(&d_total, static_cast<size_t>(nb) * 8)))
+        return cleanup(rc);
+    for (int64_t b0 = 0; b0 < r->B; b0 += nb) {
+        const int n = static_cast<int>(std::min<int64_t>(nb, r->B - b0));
+        cudaError_t e = cudaMemsetAsync(leafsum, 0, per_block * n, st);
+        if (e == cudaSuccess)
+            e = launch_index_sums(r->view(), r->tables(), r->d_idx_slots, L, b0, n, leafsum, r->d_status, r->n_sm, st);
+        if (e == cudaSuccess)
+            e = launch_index_size(leafsum, r->d_idx_root_leaf0, L, G, n, r->d_idx_desc + b0 * G, d_total, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(total.data(), d_total, static_cast<size_t>(n) * 8, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess)
+            e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess)
+            return cleanup(cuda_status(e));
+        for (int i = 0; i < n; ++i)
+            if ((rc = place_index(r, total[i], base[b0 + i])))
+                return cleanup(rc);
+        e = cudaMemcpyAsync(r->d_idx_base + b0, base.data() + b0, static_cast<size_t>(n) * 8, cudaMemcpyHostToDevice,
+                            st);
+        if (e == cudaSuccess)
+            e = launch_index_pack(leafsum, r->d_idx_root_leaf0, L, G, b0, n, r->d_idx_desc, r->d_idx_base, st);
+        if (e != cudaSuccess)
+            return cleanup(cuda_status(e));
+    }
+    // malformed streams met while summing make the index unusable
+    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+    if ((rc = bounded_wait(st)))
+        return cleanup(rc);
+    if (r->h_status->flags) {
+        rc = report_errors(r, st);
+        return cleanup(rc ? rc : QEM_ERR_MALFORMED);
+    }
+    r->has_index = true;
+    return cleanup(QEM_OK);
 }
 
 }  // namespace
@@ -592,6 +804,27 @@ int qem_decode_blocks(qem_resident *r, int64_t first, int64_t n, void *d_out, in
     return QEM_OK;
 }
 
+int qem_decode_blocks_amplitude(qem_resident *r, int64_t first, int64_t n, void *d_counts, float *d_amp,
+                                int32_t wait, void *stream)
+{
+    if (!r || !d_amp || (reinterpret_cast<uintptr_t>(d_amp) & 3u))
+        return QEM_ERR_ARG;
+    int rc = qem_decode_blocks(r, first, n, d_counts, 0, stream);
+    if (rc)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n > 0)
+        QEM_CK(launch_amplitude(d_counts, r->w, d_amp, static_cast<long long>(n) * kScans * r->P, st));
+    if (wait) {
+        QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+        rc = bounded_wait(st);
+        if (rc)
+            return rc;
+        return report_errors(r, st);
+    }
+    return QEM_OK;
+}
+
 int qem_finish(qem_resident *r, void *stream)
 {
     if (!r)
@@ -629,12 +862,18 @@ int qem_info(const qem_resident *r, qem_info_t *o)
     for (auto &kv : r->baselines)
         dev += r->P + static_cast<uint64_t>((r->B + kv.first - 1) / kv.first) * kScans * 8;
     dev += sizeof(HostTables);
+    if (r->has_index)
+        dev += r->idx_bytes + static_cast<uint64_t>(r->B) * (r->idx_L + r->idx_R) * 4 + r->B * 8 +
+               static_cast<uint64_t>(r->idx_L) * 64 * 4 + (r->idx_R + 1) * 4 + (r->idx_L + r->idx_R) * 4;
     o->device_bytes = dev;
     for (int i = 0; i < 5; ++i)
         o->form_count[i] = r->form_count[i];
     for (int m = 0; m < kModels; ++m)
         o->model_count[m] = r->model_count[m];
     o->n_arenas = static_cast<int32_t>(r->arenas.size());
+    o->index_bytes = r->has_index ? r->idx_bytes : 0;
+    o->index_leaves = r->has_index ? r->idx_L : 0;
+    o->index_roots = r->has_index ? r->idx_R : 0;
     return QEM_OK;
 }
 
@@ -788,6 +1027,65 @@ int qem_import(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t d
         return fail(cuda_status(e));
     r->B_done = r->B;
     *out = r;
+    return QEM_OK;
+}
+
+int qem_build_index(qem_resident *r, double center_row, double center_col, void *stream)
+{
+    if (!r || !std::isfinite(center_row) || !std::isfinite(center_col))
+        return QEM_ERR_ARG;
+    if (r->B_done != r->B)
+        return QEM_ERR_STATE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // queries in flight on this stream read the old index
+    QEM_CK(cudaStreamSynchronize(st));
+    return build_index(r, center_row, center_col, st);
+}
+
+int qem_drop_index(qem_resident *r, void *stream)
+{
+    if (!r)
+        return QEM_ERR_ARG;
+    QEM_CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    drop_index(r);
+    return QEM_OK;
+}
+
+int qem_index_layout(const qem_resident *r, uint32_t *h_slots, int32_t *h_root_leaf0, int32_t *n_leaves,
+                     int32_t *n_roots)
+{
+    if (!r)
+        return QEM_ERR_ARG;
+    if (!r->has_index)
+        return QEM_ERR_STATE;
+    if (n_leaves)
+        *n_leaves = r->idx_L;
+    if (n_roots)
+        *n_roots = r->idx_R;
+    if (h_slots)
+        QEM_CK(cudaMemcpy(h_slots, r->d_idx_slots, static_cast<size_t>(r->idx_L) * 64 * 4, cudaMemcpyDeviceToHost));
+    if (h_root_leaf0)
+        QEM_CK(cudaMemcpy(h_root_leaf0, r->d_idx_root_leaf0, static_cast<size_t>(r->idx_R + 1) * 4,
+                          cudaMemcpyDeviceToHost));
+    return QEM_OK;
+}
+
+int qem_export_valid(const qem_resident *r, uint8_t *h_valid)
+{
+    if (!r || !h_valid)
+        return QEM_ERR_ARG;
+    std::memcpy(h_valid, r->h_valid.data(), r->h_valid.size());
+    return QEM_OK;
+}
+
+int qem_index_desc(const qem_resident *r, uint32_t *h_desc)
+{
+    if (!r || !h_desc)
+        return QEM_ERR_ARG;
+    if (!r->has_index)
+        return QEM_ERR_STATE;
+    QEM_CK(cudaMemcpy(h_desc, r->d_idx_desc, static_cast<size_t>(r->B) * (r->idx_L + r->idx_R) * 4,
+                      cudaMemcpyDeviceToHost));
     return QEM_OK;
 }
 

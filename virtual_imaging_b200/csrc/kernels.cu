@@ -919,7 +919,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
     // the decode that follows may start its prologue (table copy) now; it
     // waits for this grid's completion before it reads anything written here
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (blockIdx.x == 0 && threadIdx.x < 2)
+    if (blockIdx.x == 0 && threadIdx.x < 4)
         count_next[threadIdx.x] = 0u;
     if (static_cast<int>(blockIdx.x) < n_list_blocks) {
         constexpr int NW = kPlanThreads / 32;
@@ -1017,6 +1017,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     }
     const uint32_t e = listed ? __ldg(list + idx) : 0u;
     const int p = static_cast<int>(e & 0x7FFFFFFFu);
+    listed = listed && p < v.P;     // the index build's lists hold padding slots (p >= P)
     const bool neg = DELTA && (e >> 31) != 0u;
     Stream S;
     S.form = kEmpty;
@@ -1062,7 +1063,11 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     // warps whose lanes hold only empty, sparse or run-decoded streams skip the per-scan loop
     const bool dense = __any_sync(kFull, dense_lane);
 
-    if (W == 1) {
+    // A uint16 warp whose dense lanes all carry values of at most 255 (paired
+    // streams without base or raw bits, whose values are table symbols, and
+    // small constants) takes the packed uint8 path as well.
+    const bool packed = W == 1 || __all_sync(kFull, !dense_lane || fast || (S.form == kConstant && S.c <= 255u));
+    if (packed) {
         // counts fit 16-bit halves: pack scans (2j, 2j+1) into one word; a
         // leaving pixel contributes 255 - v per half and the warp subtracts
         // 255 x (number of such lanes) afterwards.
@@ -1087,7 +1092,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj)
                     pk[jj] = vv[2 * jj] | (vv[2 * jj + 1] << 16);
-            } else if (S.form == kLiteral) {
+            } else if (W == 1 && S.form == kLiteral) {
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     if (S.bt.n < 16)
@@ -1218,6 +1223,79 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     }
 }
 
+// One index task: items [c * K, ...) of the item list, for block
+// b (output row `row`).  Item: bit 31 = subtract, bit 30 = root level, bits
+// 0-29 = group number within its level.  A group's 512 sums are stored with
+// one width per (block, group) (desc bits 30-31: 0 = all zero, 1/2/3 = 1, 2
+// or 4 bytes per sum; bits 0-29 = byte offset in the block's index bytes).
+// Lane l adds the sums of scans l, l + 32, ..., l + 480 (coalesced reads).
+// A task's partial sums stay below 2^31 in magnitude (K = 32 groups of at
+// most 1024 8-bit counts, or 16 groups of 16-bit counts), so a 64-bit output
+// takes them sign-extended.
+template <int W>
+__device__ __forceinline__ void index_task(const IndexView &ix, long long b, int c, uint32_t n_it, long long row,
+                                           void *out, void *keep, int out_bytes, int lane)
+{
+    constexpr uint32_t K = W == 1 ? 32u : 16u;      // items per task
+    uint32_t acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        acc[j] = 0u;
+    // lane i fetches item i of the task and its descriptor: one round trip
+    // for all of them
+    const uint32_t i0 = static_cast<uint32_t>(c) * K;
+    const uint32_t cnt = min(K, n_it - i0);
+    uint32_t my_it = 0u, my_d = 0u;
+    if (static_cast<uint32_t>(lane) < cnt) {
+        my_it = __ldg(ix.items + i0 + lane);
+        const int g = static_cast<int>(my_it & 0x3FFFFFFFu) + (((my_it >> 30) & 1u) ? ix.L : 0);
+        my_d = __ldg(ix.desc + static_cast<long long>(b) * ix.G + g);
+    }
+    const unsigned long long base = __ldg(ix.base + b);
+    for (uint32_t i = 0; i < cnt; ++i) {
+        const uint32_t d = __shfl_sync(kFull, my_d, static_cast<int>(i));
+        const uint32_t it = __shfl_sync(kFull, my_it, static_cast<int>(i));
+        const uint32_t code = d >> 30;
+        if (code == 0u)
+            continue;
+        const unsigned long long a = base + (d & 0x3FFFFFFFu);
+        const uint32_t sgn = (it >> 31) ? 0xFFFFFFFFu : 0u;     // v -> (v ^ sgn) - sgn negates
+        uint32_t v[16];
+        if (code == 1u) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                v[j] = __ldg(reinterpret_cast<const uint8_t *>(a) + lane + 32 * j);
+        } else if (code == 2u) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                v[j] = __ldg(reinterpret_cast<const uint16_t *>(a) + lane + 32 * j);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                v[j] = __ldg(reinterpret_cast<const uint32_t *>(a) + lane + 32 * j);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            acc[j] += (v[j] ^ sgn) - sgn;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        if (acc[j] == 0u)
+            continue;
+        const long long o = row * kScans + lane + 32 * j;
+        if (out_bytes == 4) {
+            atomicAdd(reinterpret_cast<unsigned int *>(out) + o, acc[j]);
+            if (keep)
+                atomicAdd(reinterpret_cast<unsigned int *>(keep) + o, acc[j]);
+        } else {
+            const unsigned long long wide = static_cast<unsigned long long>(static_cast<long long>(static_cast<int>(acc[j])));
+            atomicAdd(reinterpret_cast<unsigned long long *>(out) + o, wide);
+            if (keep)
+                atomicAdd(reinterpret_cast<unsigned long long *>(keep) + o, wide);
+        }
+    }
+}
+
 constexpr int kMaxSlots = 8;    // block rows one CTA range may touch (shared accumulators)
 
 template <int W, int THREADS, bool DELTA>
@@ -1228,7 +1306,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
                                                              const uint32_t *__restrict__ count, int stride,
                                                              long long rows, void *__restrict__ out,
                                                              void *__restrict__ keep, int out_bytes,
-                                                             DevStatus *__restrict__ st)
+                                                             IndexView ix, DevStatus *__restrict__ st)
 {
     constexpr int MAXW = THREADS / 32;
     // shared memory: one 4 KB table per model (the run tables of the first
@@ -1257,6 +1335,22 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     const uint32_t n_l = __ldg(count + 1);    // light entries, list[P - n_l, P)
     const long long tiles = ((n + 31u) >> 5) + ((n_l + 31u) >> 5);
     const long long total = rows * tiles;
+    const int warp0 = threadIdx.x >> 5, lane0 = threadIdx.x & 31;
+    if (ix.desc != nullptr) {
+        // index items (whole groups inside the mask, or inside its change):
+        // K per task (32, or 16 for 16-bit counts), each lane adding the groups' stored sums of
+        // scans lane, lane + 32, ...; the sums go straight to the output
+        const uint32_t n_it = __ldg(count + 2);
+        constexpr uint32_t K = W == 1 ? 32u : 16u;
+        const long long chunks = (n_it + K - 1) / K;
+        const long long itotal = rows * chunks;
+        const long long I0 = itotal * blockIdx.x / gridDim.x, I1 = itotal * (blockIdx.x + 1) / gridDim.x;
+        for (long long t = I0 + warp0; t < I1; t += MAXW) {
+            const long long row = t / chunks;
+            const int c = static_cast<int>(t - row * chunks);
+            index_task<W>(ix, row * stride, c, n_it, row, out, keep, out_bytes, lane0);
+        }
+    }
     // Each CTA owns one contiguous share [T0, T1) of the tasks (row-major:
     // row, then tile); its warps take the next task from a shared counter as
     // they finish, with no barrier between tasks.  Scan sums of a row gather
@@ -1476,6 +1570,16 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
     }
 }
 
+// float32 square-root amplitude of decoded counts (the feed's second output;
+// sqrtf is the correctly rounded square root)
+template <typename T>
+__global__ void k_amplitude(const T *__restrict__ in, float *__restrict__ out, long long n)
+{
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        out[i] = sqrtf(static_cast<float>(in[i]));
+}
+
 int sm_count()
 {
     static int n = 0;
@@ -1490,6 +1594,256 @@ int sm_count()
 }
 
 constexpr size_t kTableBytes = static_cast<size_t>(kModels) * kStates * sizeof(uint32_t);
+
+// ---------------------------------------------------------------------------
+// interaction index: build
+// ---------------------------------------------------------------------------
+// Pass 1: every stream of nblk blocks from block b0 is decoded and its counts
+// added per scan into its leaf's sums, leafsum[bb][leaf][512] (global, zeroed
+// by the caller).  The list is the polar slot order (64 slots per leaf,
+// padding slots hold P); a task is one block and 32 slots (half a leaf).
+template <int W>
+__global__ void __launch_bounds__(768, 1) k_index_sums(View v, const uint32_t *__restrict__ dec_g,
+                                                      const uint32_t *__restrict__ runs_g, uint32_t skip_models,
+                                                      int skip_count, const uint32_t *__restrict__ slots, int L,
+                                                      long long b0, int nblk, uint32_t *__restrict__ leafsum,
+                                                      DevStatus *__restrict__ st)
+{
+    constexpr int THREADS = 768, MAXW = THREADS / 32;
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *s_dec = smem;
+    uint32_t *s_stage = smem + kModels * kStates;
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ uint32_t s_cnt[2];
+    if (threadIdx.x == 0)
+        tables_start(&s_bar, s_dec + skip_count * kStates, dec_g + skip_count * kStates,
+                     static_cast<uint32_t>(kModels - skip_count) * kStates * 4u, s_dec, runs_g,
+                     static_cast<uint32_t>(skip_count) * kStates * 4u);
+    if (threadIdx.x < 2)
+        s_cnt[threadIdx.x] = 0u;
+    __syncthreads();
+    bool ready = false;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long tiles = 2ll * L;
+    const long long total = tiles * nblk;
+    for (long long t = static_cast<long long>(blockIdx.x) * MAXW + warp; t < total;
+         t += static_cast<long long>(gridDim.x) * MAXW) {
+        const long long bb = t / tiles;
+        const int tile = static_cast<int>(t - bb * tiles);
+        decode_task<W, false>(v, s_dec, dec_g, skip_models, slots, static_cast<uint32_t>(64 * L), 0u, tile, b0 + bb,
+                              leafsum + (bb * L + tile / 2) * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready,
+                              lane, st);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !ready)
+        tables_wait(&s_bar, st);
+}
+
+// The 512 sums of group g of block bb: a leaf's from leafsum; a root's as
+// the sum of its leaves [root_leaf0[r], root_leaf0[r+1]).
+__device__ __forceinline__ uint32_t group_sum(const uint32_t *leafsum, const int *root_leaf0, int L, long long bb,
+                                              int g, int sc)
+{
+    if (g < L)
+        return leafsum[(bb * L + g) * kScans + sc];
+    const int r = g - L;
+    uint32_t t = 0;
+    for (int l = root_leaf0[r]; l < root_leaf0[r + 1]; ++l)
+        t += leafsum[(bb * L + l) * kScans + sc];
+    return t;
+}
+
+// Pass 2 (one CTA per block): each group's width code from its largest sum,
+// then the byte offsets (exclusive scan over the groups) into desc[bb][G];
+// the block's total bytes into total[bb].
+__global__ void __launch_bounds__(1024) k_index_size(const uint32_t *__restrict__ leafsum,
+                                                    const int *__restrict__ root_leaf0, int L, int G,
+                                                    uint32_t *__restrict__ desc, unsigned long long *__restrict__ total)
+{
+    extern __shared__ uint32_t s_sz[];     // [G] bytes of each group
+    const long long bb = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int g = warp; g < G; g += nw) {
+        uint32_t mx = 0;
+        for (int sc = lane; sc < kScans; sc += 32)
+            mx = max(mx, group_sum(leafsum, root_leaf0, L, bb, g, sc));
+        mx = __reduce_max_sync(kFull, mx);
+        if (lane == 0)
+            s_sz[g] = mx == 0u ? 0u : (mx <= 0xFFu ? 1u : (mx <= 0xFFFFu ? 2u : 3u));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long off = 0;
+        for (int g = 0; g < G; ++g) {
+            const uint32_t code = s_sz[g];
+            desc[bb * G + g] = static_cast<uint32_t>(off) | (code << 30);
+            off += code == 0u ? 0u : (static_cast<unsigned long long>(kScans) << (code - 1u));
+        }
+        total[bb] = off;
+    }
+}
+
+// Pass 3: write each group's sums at its width to base[b0 + bb] + offset.
+__global__ void __launch_bounds__(512) k_index_pack(const uint32_t *__restrict__ leafsum,
+                                                   const int *__restrict__ root_leaf0, int L, int G, long long b0,
+                                                   const uint32_t *__restrict__ desc_all,
+                                                   const unsigned long long *__restrict__ base)
+{
+    const long long bb = blockIdx.y;
+    const int g = blockIdx.x;
+    const uint32_t d = desc_all[(b0 + bb) * G + g];
+    const uint32_t code = d >> 30;
+    if (code == 0u)
+        return;
+    const unsigned long long a = base[b0 + bb] + (d & 0x3FFFFFFFu);
+    for (int sc = threadIdx.x; sc < kScans; sc += blockDim.x) {
+        const uint32_t val = group_sum(leafsum, root_leaf0, L, bb, g, sc);
+        if (code == 1u)
+            reinterpret_cast<uint8_t *>(a)[sc] = static_cast<uint8_t>(val);
+        else if (code == 2u)
+            reinterpret_cast<uint16_t *>(a)[sc] = static_cast<uint16_t>(val);
+        else
+            reinterpret_cast<uint32_t *>(a)[sc] = val;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// interaction index: plan (one CTA per root, one warp per leaf)
+// ---------------------------------------------------------------------------
+// A leaf whose every pixel is in the mask (full query), or whose every pixel
+// enters, or every pixel leaves, the mask (delta) becomes one index item; a
+// root whose leaves all do so in the same direction becomes one root item
+// instead.  The remaining masked (changed) pixels go to the residual list as
+// in k_plan.  The counts are count[0] heavy, count[1] light, count[2] items.
+__global__ void __launch_bounds__(512) k_plan_index(const uint8_t *__restrict__ mask,
+                                                   const uint8_t *__restrict__ pclass,
+                                                   uint8_t *__restrict__ base_mask, int P, int mode,
+                                                   const uint32_t *__restrict__ slots,
+                                                   const int *__restrict__ root_leaf0, int R,
+                                                   uint32_t *__restrict__ list, uint32_t *__restrict__ items,
+                                                   uint32_t *__restrict__ count, uint32_t *__restrict__ count_next,
+                                                   uint4 *__restrict__ out, uint4 *__restrict__ keep, long long n_vec)
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x < 4)
+        count_next[threadIdx.x] = 0u;
+    if (static_cast<int>(blockIdx.x) < R) {
+        constexpr int NW = 16;
+        __shared__ int s_state[NW];            // per leaf: 1 all enter/in, 2 all leave, 0 otherwise, -1 none
+        __shared__ uint32_t s_h[NW], s_l[NW], s_at[2];
+        const int r = blockIdx.x;
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int l0 = root_leaf0[r], nl = root_leaf0[r + 1] - l0;
+        const int leaf = l0 + warp;
+        bool emit[2] = {false, false}, light[2] = {false, false};
+        uint32_t entry[2] = {0u, 0u};
+        int state = -1;
+        if (warp < nl) {
+            bool all_in = true, all_out = true;
+            const uint2 pp = reinterpret_cast<const uint2 *>(slots + leaf * 64)[lane];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t p = k ? pp.y : pp.x;
+                if (p >= static_cast<uint32_t>(P))
+                    continue;
+                const uint8_t mk = mask[p];
+                const bool nw = mk != 0;
+                const bool od = base_mask[p] != 0;
+                bool add, rem;
+                if (mode == 0) {
+                    add = nw;
+                    rem = false;
+                } else {
+                    add = nw && !od;
+                    rem = !nw && od;
+                }
+                all_in = all_in && add;
+                all_out = all_out && rem;
+                emit[k] = add || rem;
+                entry[k] = p | (rem ? 0x80000000u : 0u);
+                light[k] = pclass[p] != 0;
+                base_mask[p] = mk;
+            }
+            all_in = __all_sync(kFull, all_in);
+            all_out = __all_sync(kFull, all_out) && mode == 1;
+            state = all_in ? 1 : (all_out ? 2 : 0);
+        }
+        if (lane == 0)
+            s_state[warp] = state;
+        __syncthreads();
+        // the root as one item when all its leaves go the same way
+        int rs = s_state[0];
+        for (int k = 1; k < nl; ++k)
+            rs = s_state[k] == rs ? rs : 0;
+        const bool root_item = nl > 0 && rs > 0;
+        if (state > 0 || root_item) {
+            emit[0] = emit[1] = false;        // covered by an index item
+        }
+        // index items: one reservation per CTA (the root, or its whole leaves in order)
+        if (threadIdx.x == 0) {
+            if (root_item) {
+                items[atomicAdd(count + 2, 1u)] = static_cast<uint32_t>(r) | (1u << 30) | (rs == 2 ? 0x80000000u : 0u);
+            } else {
+                uint32_t nf = 0;
+                for (int k = 0; k < nl; ++k)
+                    nf += s_state[k] > 0;
+                if (nf) {
+                    uint32_t at = atomicAdd(count + 2, nf);
+                    for (int k = 0; k < nl; ++k)
+                        if (s_state[k] > 0)
+                            items[at++] = static_cast<uint32_t>(l0 + k) | (s_state[k] == 2 ? 0x80000000u : 0u);
+                }
+            }
+        }
+        // residual pixels: block-level reservations per class, as in k_plan
+        uint32_t nh = 0, nlt = 0;
+        unsigned bh[2], bl[2];
+        for (int k = 0; k < 2; ++k) {
+            bh[k] = __ballot_sync(kFull, emit[k] && !light[k]);
+            bl[k] = __ballot_sync(kFull, emit[k] && light[k]);
+            nh += __popc(bh[k]);
+            nlt += __popc(bl[k]);
+        }
+        if (lane == 0) {
+            s_h[warp] = nh;
+            s_l[warp] = nlt;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t th = 0, tl = 0;
+            for (int w = 0; w < NW; ++w) {
+                const uint32_t a = s_h[w], c = s_l[w];
+                s_h[w] = th;
+                s_l[w] = tl;
+                th += a;
+                tl += c;
+            }
+            s_at[0] = th ? atomicAdd(count, th) : 0u;
+            s_at[1] = tl ? atomicAdd(count + 1, tl) : 0u;
+        }
+        __syncthreads();
+        const unsigned below = (1u << lane) - 1u;
+        uint32_t oh = s_at[0] + s_h[warp], ol = s_at[1] + s_l[warp];
+        for (int k = 0; k < 2; ++k) {
+            if (emit[k] && !light[k])
+                list[oh + __popc(bh[k] & below)] = entry[k];
+            if (emit[k] && light[k])
+                list[P - 1 - (ol + __popc(bl[k] & below))] = entry[k];
+            oh += __popc(bh[k]);
+            ol += __popc(bl[k]);
+        }
+        return;
+    }
+    const long long stride = static_cast<long long>(gridDim.x - R) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x - R) * blockDim.x + threadIdx.x; i < n_vec; i += stride) {
+        if (mode == 0) {
+            out[i] = make_uint4(0u, 0u, 0u, 0u);
+            keep[i] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            out[i] = keep[i];
+        }
+    }
+}
 
 }  // namespace
 
@@ -1573,7 +1927,8 @@ cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t
 
 template <int W, int TH, bool DELTA>
 cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride, long long rows,
-                      void *out, void *keep, int out_bytes, DevStatus *status, int n_sm, cudaStream_t st)
+                      void *out, void *keep, int out_bytes, IndexView ix, DevStatus *status, int n_sm,
+                      cudaStream_t st)
 {
     // the run-decoded models are a prefix 0..k-1 (their (0,0) share falls as lambda grows)
     const int skip_count = __builtin_popcount(tb.skip_models);
@@ -1601,19 +1956,22 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
     cfg.attrs = at;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_decode_reduce<W, TH, DELTA>, v, tb.dec, tb.runs, tb.skip_models, skip_count,
-                              list, count, stride, rows, out, keep, out_bytes, status);
+                              list, count, stride, rows, out, keep, out_bytes, ix, status);
 }
 
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride,
                                  long long rows, void *out, int out_bytes, DevStatus *status, int n_sm,
-                                 cudaStream_t st, bool delta, void *keep)
+                                 cudaStream_t st, bool delta, void *keep, IndexView ix)
 {
     if (v.w == 1)
-        return delta ? launch_dr<1, 768, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm, st)
-                     : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm,
-                                                st);
-    return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm, st)
-                 : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, status, n_sm, st);
+        return delta ? launch_dr<1, 768, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
+                                               n_sm, st)
+                     : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
+                                                n_sm, st);
+    return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
+                                           st)
+                 : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
+                                            st);
 }
 
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,
@@ -1638,6 +1996,72 @@ cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n
         }
         k_decode_blocks<2><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amplitude(const void *counts, int w, float *amp, long long n, cudaStream_t st)
+{
+    long long grid = (n + 255) / 256;
+    grid = grid < 1 ? 1 : (grid > 16ll * sm_count() ? 16ll * sm_count() : grid);
+    if (w == 1)
+        k_amplitude<uint8_t><<<static_cast<int>(grid), 256, 0, st>>>(static_cast<const uint8_t *>(counts), amp, n);
+    else
+        k_amplitude<uint16_t><<<static_cast<int>(grid), 256, 0, st>>>(static_cast<const uint16_t *>(counts), amp, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_index_sums(View v, Tables tb, const uint32_t *slots, int L, long long b0, int nblk,
+                              uint32_t *leafsum, DevStatus *status, int n_sm, cudaStream_t st)
+{
+    const int skip_count = __builtin_popcount(tb.skip_models);
+    const size_t smem = kTableBytes + 24 * 16 * sizeof(uint32_t);
+    static int attr_dev[2] = {-1, -1};
+    const int wi = v.w == 1 ? 0 : 1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev[wi] != dev) {
+        const cudaError_t e = v.w == 1 ? cudaFuncSetAttribute(k_index_sums<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                              static_cast<int>(smem))
+                                       : cudaFuncSetAttribute(k_index_sums<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                              static_cast<int>(smem));
+        if (e != cudaSuccess)
+            return e;
+        attr_dev[wi] = dev;
+    }
+    if (v.w == 1)
+        k_index_sums<1><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, slots, L, b0, nblk,
+                                                  leafsum, status);
+    else
+        k_index_sums<2><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, slots, L, b0, nblk,
+                                                  leafsum, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_index_size(const uint32_t *leafsum, const int *root_leaf0, int L, int G, int nblk, uint32_t *desc,
+                              unsigned long long *total, cudaStream_t st)
+{
+    k_index_size<<<nblk, 1024, static_cast<size_t>(G) * 4, st>>>(leafsum, root_leaf0, L, G, desc, total);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_index_pack(const uint32_t *leafsum, const int *root_leaf0, int L, int G, long long b0, int nblk,
+                              const uint32_t *desc_all, const unsigned long long *base, cudaStream_t st)
+{
+    k_index_pack<<<dim3(G, nblk), 512, 0, st>>>(leafsum, root_leaf0, L, G, b0, desc_all, base);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_plan_index(const uint8_t *mask, const uint8_t *pclass, uint8_t *base_mask, int P, int mode,
+                              const uint32_t *slots, const int *root_leaf0, int R, uint32_t *list, uint32_t *items,
+                              uint32_t *count, uint32_t *count_next, void *out, void *keep, long long n_elems,
+                              int out_bytes, cudaStream_t st)
+{
+    const long long n_vec = n_elems * out_bytes / 16;
+    int fill = static_cast<int>((n_vec + 512 * 4 - 1) / (512 * 4));
+    fill = fill < 1 ? 1 : (fill > 4 * sm_count() ? 4 * sm_count() : fill);
+    k_plan_index<<<R + fill, 512, 0, st>>>(mask, pclass, base_mask, P, mode, slots, root_leaf0, R, list, items,
+                                           count, count_next, static_cast<uint4 *>(out), static_cast<uint4 *>(keep),
+                                           n_vec);
     return cudaGetLastError();
 }
 

@@ -90,6 +90,17 @@ struct View {
     long long B;
 };
 
+// Interaction index of a resident (absent when desc is null): per block, the
+// 512 per-scan sums of each of G = L + R pixel groups (L leaves of at most 64
+// pixels, R roots of at most 16 leaves), each group stored at one width.
+struct IndexView {
+    const uint32_t *desc;                 // [B][G]: bits 0-29 byte offset, 30-31 width code
+    const unsigned long long *base;       // [B] device address of each block's index bytes
+    const uint32_t *items;                // the query's index items (written by the plan)
+    int L;
+    int G;
+};
+
 const HostTables &host_tables();          // built once per process (tables.cu)
 
 // What the allocation-free masked sum needs from a resident (api.cu).
@@ -130,11 +141,25 @@ cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t
                         uint8_t *base_mask, int P, int mode, uint32_t *list, uint32_t *count,
                         uint32_t *count_next, void *out, void *keep, long long n_elems, int out_bytes,
                         cudaStream_t st);
-// keep (may be null): a second image that receives the same additions as out
+// keep (may be null): a second image that receives the same additions as out;
+// ix.desc null: no index items (count[2] is not read)
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count,
                                  int stride, long long rows, void *out, int out_bytes,
                                  DevStatus *status, int n_sm, cudaStream_t st, bool delta = false,
-                                 void *keep = nullptr);
+                                 void *keep = nullptr, IndexView ix = IndexView{nullptr, nullptr, nullptr, 0, 0});
+cudaError_t launch_amplitude(const void *counts, int w, float *amp, long long n, cudaStream_t st);
+// interaction index build (leafsum zeroed by the caller: [nblk][L][512] u32)
+cudaError_t launch_index_sums(View v, Tables tb, const uint32_t *slots, int L, long long b0, int nblk,
+                              uint32_t *leafsum, DevStatus *status, int n_sm, cudaStream_t st);
+cudaError_t launch_index_size(const uint32_t *leafsum, const int *root_leaf0, int L, int G, int nblk, uint32_t *desc,
+                              unsigned long long *total, cudaStream_t st);
+cudaError_t launch_index_pack(const uint32_t *leafsum, const int *root_leaf0, int L, int G, long long b0, int nblk,
+                              const uint32_t *desc_all, const unsigned long long *base, cudaStream_t st);
+// plan over the polar layout: residual list + index items (count[2])
+cudaError_t launch_plan_index(const uint8_t *mask, const uint8_t *pclass, uint8_t *base_mask, int P, int mode,
+                              const uint32_t *slots, const int *root_leaf0, int R, uint32_t *list, uint32_t *items,
+                              uint32_t *count, uint32_t *count_next, void *out, void *keep, long long n_elems,
+                              int out_bytes, cudaStream_t st);
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out,
                                  DevStatus *status, cudaStream_t st);
 
