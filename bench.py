@@ -313,6 +313,7 @@ def run_profile_case(dev, torch, V):
     res, buf, t_enc = build_resident(w, dev, torch, V)
     del buf
     torch.cuda.empty_cache()
+    res.build_index((w.det_rows // 2, w.det_cols // 2))
     out = torch.empty((w.n_blocks, 512), dtype=V.out_dtype(32), device=dev)
     bf = torch.from_numpy(w.masks["bf"]).to(dev)
     adf = torch.from_numpy(w.masks["adf"]).to(dev)
@@ -336,6 +337,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="c4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--saved-form", default=None, metavar="PATH",
+                    help="also time writing the resident's saved form to PATH and reopening it")
     ap.add_argument("--no-index", action="store_true",
                     help="query without the interaction index (every masked pixel decoded)")
     ap.add_argument("--profile", action="store_true", help="bounded case for ncu captures")
@@ -521,6 +524,22 @@ def main():
     te = f0.elapsed_time(f1) / 1e3
     te = max_over_ranks(te, device=dev)
 
+    saved = None
+    if args.saved_form:
+        torch.cuda.synchronize()
+        s0 = time.perf_counter()
+        res.save(args.saved_form)
+        s1 = time.perf_counter()
+        back = V.Resident.load(args.saved_form)
+        torch.cuda.synchronize()
+        s2 = time.perf_counter()
+        fbytes = os.path.getsize(args.saved_form)
+        same = all(np.array_equal(a, b) for b0 in (0, w.n_blocks - 1)
+                   for a, b in zip(res.export_block(b0), back.export_block(b0)))
+        back.free()
+        os.remove(args.saved_form)
+        saved = {"file_bytes": fbytes, "save_s": s1 - s0, "load_s": s2 - s1, "blocks_checked_equal": same}
+
     # per-query breakdown (separate, untimed for `value`)
     lens = stream_lengths(res, w)
     idx = None
@@ -587,6 +606,7 @@ def main():
                    "hbm_frac": ((w.raw_bytes + info["payload_bytes"] + info["group_bytes"]) / enc_s / 1e9 / hbm)
                    if enc_s else None},
         "index": index,
+        "saved_form": saved,
         "decode_blocks": {"blocks": nd, "s": dec_s, "gcounts_per_s": nd * 512 * w.n_pixels / dec_s / 1e9,
                           "exact": ok_frames},
         "resident": {"payload_bytes": info["payload_bytes"], "forms": info["form_count"],
