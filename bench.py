@@ -524,6 +524,25 @@ def main():
     te = f0.elapsed_time(f1) / 1e3
     te = max_over_ranks(te, device=dev)
 
+    # fused moments (centre-of-mass numerators and denominator) over the bright-field
+    # disk and the annulus, stride 1: every masked pixel decoded, 10 back to back
+    rr, cc = np.divmod(np.arange(w.n_pixels), w.det_cols)
+    wts = torch.from_numpy(np.stack([rr - w.det_rows // 2, cc - w.det_cols // 2]).astype(np.int32)).to(dev)
+    mom_out = torch.empty((3, w.n_blocks, 512), dtype=torch.int64, device=dev)
+    mom = {}
+    for name in ("bf", "adf"):
+        md = torch.from_numpy(w.masks[name].astype(np.uint8)).to(dev)
+        res.masked_moments(md, wts, out=mom_out)
+        torch.cuda.synchronize()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record()
+        for _ in range(10):
+            res.masked_moments(md, wts, out=mom_out, wait=False)
+        m1.record()
+        torch.cuda.synchronize()
+        res.finish()
+        mom[f"{name}_k1_ms"] = m0.elapsed_time(m1) / 10
+
     saved = None
     if args.saved_form:
         torch.cuda.synchronize()
@@ -607,6 +626,7 @@ def main():
                    if enc_s else None},
         "index": index,
         "saved_form": saved,
+        "moments": mom,
         "decode_blocks": {"blocks": nd, "s": dec_s, "gcounts_per_s": nd * 512 * w.n_pixels / dec_s / 1e9,
                           "exact": ok_frames},
         "resident": {"payload_bytes": info["payload_bytes"], "forms": info["form_count"],

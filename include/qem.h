@@ -218,6 +218,22 @@ int qem_load(const char *path, void *stream, qem_resident **out);
  * the resident has no index. */
 int qem_index_desc(const qem_resident *res, uint32_t *h_desc);
 
+/* Masked moments (the pages' fused CoM/DPC moment reduction: an exact
+ * integer numerator and denominator before the float divide): for each
+ * touched block row (blocks 0, k, 2k, ...) and scan, over the pixels with
+ * mask && valid,
+ *   d_out[0][row][scan] = sum x * d_weights[p]            (e.g. row offset)
+ *   d_out[1][row][scan] = sum x * d_weights[n_pixels + p] (e.g. column offset)
+ *   d_out[2][row][scan] = sum x
+ * as int64 (caller-owned, 8-byte aligned, 3 * ceil(B/k) * 512 values).
+ * d_weights: device int32 [2][n_pixels], each |w| <= 262143 (larger weights
+ * give wrong sums, not a fault).  Centre of mass = d_out[0] / d_out[2];
+ * a segmented DPC signal uses +-1 weights.  Every masked pixel is decoded
+ * (the interaction index holds no weighted sums); stride baselines are not
+ * touched.  Same wait rule and errors as qem_masked_sum. */
+int qem_masked_moments(qem_resident *res, const uint8_t *d_mask, const int32_t *d_weights, int32_t block_stride,
+                       int64_t *d_out, int32_t wait, void *stream);
+
 /* Block decode plus amplitude (page "Operation pipeline" step 6: the feed's
  * "counts plus float32 sqrt amplitude"): as qem_decode_blocks into d_counts,
  * then d_amp (float32, same [n_blocks*512][pixels] shape, 4-byte aligned)

@@ -7,8 +7,9 @@ imports it.
 
 Two layers:
 
-* plain definitions in NumPy (exact integer arithmetic, uint64):
-  :func:`dense_masked_sum`, :func:`dense_delta`, :func:`dense_decode_blocks` --
+* plain definitions in NumPy (exact integer arithmetic, uint64 / int64):
+  :func:`dense_masked_sum`, :func:`dense_delta`, :func:`dense_decode_blocks`,
+  :func:`dense_masked_moments` --
   these are the results the method must reach, written out directly from the
   source page "Paired-count resident layout" (section "Operation pipeline"
   step 4: exact integer virtual images, ``block_stride=k`` touches every k-th
@@ -262,6 +263,28 @@ def dense_masked_sum(counts: np.ndarray, mask: np.ndarray, valid: np.ndarray | N
     out = np.zeros((len(rows), 512), np.uint64)
     for r, b in enumerate(rows):
         out[r] = counts[b * 512:(b + 1) * 512][:, sel].astype(np.uint64).sum(axis=1)
+    return out
+
+
+def dense_masked_moments(counts: np.ndarray, mask: np.ndarray, weights: np.ndarray,
+                         valid: np.ndarray | None = None, k: int = 1) -> np.ndarray:
+    """Plain definition of the fused moment reduction (page "Backend Optimization Matrix",
+    CoM/DPC rows: a fused moment reducer whose centre of mass is exact before the divide):
+    for each touched block row r and scan i, over the pixels p with mask & valid,
+    M[0][r][i] = sum x*w[0][p], M[1][r][i] = sum x*w[1][p], M[2][r][i] = sum x (int64)."""
+    sel = mask.astype(bool)
+    if valid is not None:
+        sel &= valid.astype(bool)
+    B = counts.shape[0] // 512
+    rows = touched_blocks(B, k)
+    w0 = weights[0][sel].astype(np.int64)
+    w1 = weights[1][sel].astype(np.int64)
+    out = np.zeros((3, len(rows), 512), np.int64)
+    for r, b in enumerate(rows):
+        x = counts[b * 512:(b + 1) * 512][:, sel].astype(np.int64)
+        out[0, r] = x @ w0
+        out[1, r] = x @ w1
+        out[2, r] = x.sum(axis=1)
     return out
 
 

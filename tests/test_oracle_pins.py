@@ -438,3 +438,44 @@ def test_delta_chain_equals_full():
         for t in range(1, len(w.drag)):
             img = O.resident_delta(enc, img, w.drag[t - 1], w.drag[t], None, k)
             assert (img == O.dense_masked_sum(x, w.drag[t], None, k)).all(), (k, t)
+
+
+def test_moments_pins():
+    """The moment definition against closed forms: unit weights give the masked sum; one lit
+    pixel per scan puts the centre of mass exactly on it; weights are linear; a pattern mirrored
+    about the centre has zero first moment; strides take the touched blocks."""
+    rng = np.random.default_rng(11)
+    R, C, scans = 9, 11, 1024
+    P = R * C
+    x = rng.integers(0, 300, size=(scans, P)).astype(np.uint16)
+    mask = (rng.random(P) < 0.6).astype(np.uint8)
+    valid = (rng.random(P) < 0.9).astype(np.uint8)
+    ones = np.ones((2, P), np.int32)
+    m = O.dense_masked_moments(x, mask, ones, valid, 1)
+    s = O.dense_masked_sum(x, mask, valid, 1).astype(np.int64)
+    assert (m[0] == s).all() and (m[1] == s).all() and (m[2] == s).all()
+    # one lit pixel per scan: CoM = its (row - r0, col - c0) exactly
+    r0, c0 = 4, 5
+    rr, cc = np.divmod(np.arange(P), C)
+    w = np.stack([rr - r0, cc - c0]).astype(np.int32)
+    lit = rng.integers(0, P, size=scans)
+    y = np.zeros((scans, P), np.uint16)
+    y[np.arange(scans), lit] = rng.integers(1, 60000, size=scans)
+    full = np.ones(P, np.uint8)
+    m = O.dense_masked_moments(y, full, w)
+    assert (m[2].reshape(-1) == y.sum(axis=1)).all()
+    assert (m[0].reshape(-1) == y.sum(axis=1).astype(np.int64) * (lit // C - r0)).all()
+    assert (m[1].reshape(-1) == y.sum(axis=1).astype(np.int64) * (lit % C - c0)).all()
+    # linear in the weights
+    w2 = rng.integers(-1000, 1000, size=(2, P)).astype(np.int32)
+    a = O.dense_masked_moments(x, mask, w, valid, 2)
+    b = O.dense_masked_moments(x, mask, w2, valid, 2)
+    c = O.dense_masked_moments(x, mask, (w + w2).astype(np.int32), valid, 2)
+    assert (c[:2] == a[:2] + b[:2]).all() and (c[2] == a[2]).all()
+    # a pattern mirrored about the centre row has zero row moment
+    z = rng.integers(0, 50, size=(scans, R, C)).astype(np.uint16)
+    z = (z + z[:, ::-1, :]).reshape(scans, P)
+    assert (O.dense_masked_moments(z, full, w)[0] == 0).all()
+    # stride k: rows of the touched blocks
+    assert (O.dense_masked_moments(x, mask, w, valid, 2)[:, 0] == O.dense_masked_moments(x, mask, w, valid, 1)[:, 0]).all()
+    assert O.dense_masked_moments(x, mask, w, valid, 3).shape == (3, 1, 512)

@@ -32,7 +32,7 @@ EXPORTS = ("qem_abi", "qem_status_string", "qem_create", "qem_encode", "qem_enco
            "qem_profile", "qem_profile_read", "qem_free", "qem_block_bytes", "qem_export_block", "qem_import",
            "qem_model_tables", "qem_generate_counts", "qem_masked_sum_noalloc", "qem_build_index",
            "qem_drop_index", "qem_index_layout", "qem_index_desc", "qem_export_valid", "qem_save", "qem_load",
-           "qem_decode_blocks_amplitude")
+           "qem_decode_blocks_amplitude", "qem_masked_moments")
 
 
 class QemError(RuntimeError):
@@ -107,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "qem_save": ([vp, ctypes.c_char_p, vp], ctypes.c_int),
         "qem_load": ([ctypes.c_char_p, vp, pp], ctypes.c_int),
         "qem_decode_blocks_amplitude": ([vp, i64, i64, vp, vp, i32, vp], ctypes.c_int),
+        "qem_masked_moments": ([vp, vp, vp, i32, vp, i32, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -248,6 +249,19 @@ class Resident:
         chosen width); calls that overlap on the GPU race on the library's fixed working memory."""
         _check(lib().qem_masked_sum_noalloc(self._h, _dev_ptr(mask), block_stride, out_bits, _dev_ptr(out),
                                             _stream(stream)), "qem_masked_sum_noalloc")
+        return out
+
+    def masked_moments(self, mask: torch.Tensor, weights: torch.Tensor, block_stride: int = 1,
+                       out: torch.Tensor | None = None, wait: bool = True, stream=None) -> torch.Tensor:
+        """int64 [3][ceil(B/k)][512]: (sum x*w0, sum x*w1, sum x) per scan over mask & valid pixels.
+        weights: int32 [2][pixels] on the device, |w| <= 262143."""
+        if out is None:
+            n_blocks = self._static()[0]
+            if block_stride < 1:
+                raise QemError(QEM_ERR_ARG, "qem_masked_moments")
+            out = torch.empty((3, -(-n_blocks // block_stride), 512), dtype=torch.int64, device=mask.device)
+        _check(lib().qem_masked_moments(self._h, _dev_ptr(mask), _dev_ptr(weights), block_stride, _dev_ptr(out),
+                                        1 if wait else 0, _stream(stream)), "qem_masked_moments")
         return out
 
     def decode_blocks(self, first: int, n: int, out: torch.Tensor | None = None, wait: bool = True,

@@ -95,6 +95,7 @@ struct qem_resident {
     uint32_t *d_idx_items = nullptr;            // [L + R] items of the current query
     std::vector<Arena> idx_arenas;
     uint64_t idx_bytes = 0;
+    uint8_t *d_mom_mask = nullptr;              // scratch mask store of the moments plan
     DevStatus *d_status = nullptr;
     DevStatus *h_status = nullptr;              // pinned
     std::map<int, Baseline> baselines;
@@ -196,6 +197,7 @@ void release(qem_resident *r)
     cudaFree(r->d_idx_desc);
     cudaFree(r->d_idx_base);
     cudaFree(r->d_idx_items);
+    cudaFree(r->d_mom_mask);
     for (auto &kv : r->baselines) {
         cudaFree(kv.second.d_mask);
         cudaFree(kv.second.d_img);
@@ -791,6 +793,44 @@ int qem_decode_blocks(qem_resident *r, int64_t first, int64_t n, void *d_out, in
         return QEM_OK;
     int rc = timed(r, QEM_K_DECODE_BLOCKS, st, [&] {
         return launch_decode_blocks(r->view(), r->tables(), first, n, d_out, r->d_status, st);
+    });
+    if (rc)
+        return rc;
+    if (wait) {
+        QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+        rc = bounded_wait(st);
+        if (rc)
+            return rc;
+        return report_errors(r, st);
+    }
+    return QEM_OK;
+}
+
+int qem_masked_moments(qem_resident *r, const uint8_t *d_mask, const int32_t *d_weights, int32_t k, int64_t *d_out,
+                       int32_t wait, void *stream)
+{
+    if (!r || !d_mask || !d_weights || !d_out || k < 1 || (reinterpret_cast<uintptr_t>(d_out) & 7u) ||
+        (reinterpret_cast<uintptr_t>(d_weights) & 3u))
+        return QEM_ERR_ARG;
+    if (r->B_done != r->B)
+        return QEM_ERR_STATE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc;
+    if (!r->d_mom_mask && (rc = dalloc(&r->d_mom_mask, static_cast<size_t>(r->P))))
+        return rc;
+    const long long rows = (r->B + k - 1) / k;
+    uint32_t *count = r->d_count + 4 * r->count_pair;
+    uint32_t *count_next = r->d_count + 4 * (r->count_pair ^ 1);
+    rc = timed(r, QEM_K_PLAN, st, [&] {
+        return launch_plan(d_mask, r->d_valid, r->d_pclass, r->d_mom_mask, r->P, 0, r->d_list, count, count_next,
+                           nullptr, nullptr, 0, 8, st);
+    });
+    if (rc)
+        return rc;
+    r->count_pair ^= 1;
+    rc = timed(r, QEM_K_DECODE_REDUCE, st, [&] {
+        return launch_moments(r->view(), r->tables(), r->d_list, count, d_weights, k, rows,
+                              reinterpret_cast<long long *>(d_out), r->d_status, st);
     });
     if (rc)
         return rc;

@@ -18,6 +18,10 @@
 #include <cstdio>
 #include <type_traits>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "qem_internal.h"
 
 namespace qem {
@@ -1476,6 +1480,173 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
 // ---------------------------------------------------------------------------
 // a7: block decode into native frames
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// masked moments (fused CoM / DPC numerators and denominator)
+// ---------------------------------------------------------------------------
+// For every touched block row and scan: sum of x * wr[p], of x * wc[p] and of
+// x over the listed pixels (the plan's list of mask && valid pixels), exact in
+// int64.  One CTA owns a row at a time (its warps take the row's tiles from a
+// shared counter), so the row is written with plain stores.  Dense forms go
+// through warp reductions of 32-bit partial sums (for 16-bit counts the value
+// is split in bytes, so every partial sum stays below 2^31 for |w| < 2^18);
+// sparse streams scatter their nonzeros into the row with shared atomics.
+// Paired streams of every model use the general decode (decode tables of all
+// 32 models in shared memory).
+template <int W>
+__global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__restrict__ dec_g,
+                                                   const uint32_t *__restrict__ list,
+                                                   const uint32_t *__restrict__ count,
+                                                   const int32_t *__restrict__ weights, int stride, long long rows,
+                                                   long long *__restrict__ out, DevStatus *__restrict__ st)
+{
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *s_dec = smem;
+    unsigned long long *s_acc = reinterpret_cast<unsigned long long *>(smem + kModels * kStates);  // [3][512]
+    __shared__ unsigned s_next;
+    for (int i = threadIdx.x; i < kModels * kStates / 4; i += blockDim.x)
+        reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
+    for (int i = threadIdx.x; i < 3 * kScans; i += blockDim.x)
+        s_acc[i] = 0ull;
+    const uint32_t n = __ldg(count), n_l = __ldg(count + 1);
+    const uint32_t tiles_h = (n + 31u) >> 5;
+    const uint32_t tiles = tiles_h + ((n_l + 31u) >> 5);
+    const int lane = threadIdx.x & 31;
+    const long long P = v.P;
+    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+        if (threadIdx.x == 0)
+            s_next = 0u;
+        __syncthreads();
+        const long long b = row * stride;
+        while (true) {
+            unsigned tile = 0;
+            if (lane == 0)
+                tile = atomicAdd(&s_next, 1u);
+            tile = __shfl_sync(kFull, tile, 0);
+            if (tile >= tiles)
+                break;
+            uint32_t idx;
+            bool listed;
+            if (tile < tiles_h) {
+                idx = tile * 32u + static_cast<uint32_t>(lane);
+                listed = idx < n;
+            } else {
+                idx = static_cast<uint32_t>(P) - n_l + (tile - tiles_h) * 32u + static_cast<uint32_t>(lane);
+                listed = idx < static_cast<uint32_t>(P);
+            }
+            const int p = listed ? static_cast<int>(__ldg(list + idx) & 0x7FFFFFFFu) : 0;
+            const long long wr = listed ? __ldg(weights + p) : 0, wc = listed ? __ldg(weights + P + p) : 0;
+            Stream S;
+            S.form = kEmpty;
+            S.model = 0;
+            S.shift = 0;
+            S.base = 0;
+            S.c = 0;
+            S.x = 0;
+            S.len = 0;
+            bool ok = listed;
+            if (ok)
+                ok = locate(v, b, p, S.s, S.len, st);
+            if (ok)
+                ok = open_stream(S, W, st);
+            if (!ok)
+                S.form = kEmpty;
+            const bool dense_lane = S.form == kPaired || S.form == kLiteral || S.form == kConstant;
+            const bool dense = __any_sync(kFull, dense_lane);
+            const uint32_t *dec = s_dec + S.model * kStates;
+            uint32_t over = 0;
+            for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
+                uint32_t vv[32];
+                if (S.form == kPaired) {
+                    paired_segment(S, dec, vv, over);
+                } else if (S.form == kLiteral) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (S.bt.n < 16)
+                            S.bt.refill();
+                        vv[i] = S.bt.get(8 * W);
+                    }
+                } else {
+                    const uint32_t c = S.form == kConstant ? S.c : 0u;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        vv[i] = c;
+                }
+                long long m0 = 0, m1 = 0, m2 = 0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int x0 = static_cast<int>(vv[i]);
+                    int a0 = __reduce_add_sync(kFull, x0);
+                    long long a1, a2;
+                    if (W == 1) {
+                        a1 = __reduce_add_sync(kFull, x0 * static_cast<int>(wr));
+                        a2 = __reduce_add_sync(kFull, x0 * static_cast<int>(wc));
+                    } else {
+                        const int lo = x0 & 0xFF, hi = x0 >> 8;
+                        a1 = static_cast<long long>(__reduce_add_sync(kFull, lo * static_cast<int>(wr))) +
+                             256ll * __reduce_add_sync(kFull, hi * static_cast<int>(wr));
+                        a2 = static_cast<long long>(__reduce_add_sync(kFull, lo * static_cast<int>(wc))) +
+                             256ll * __reduce_add_sync(kFull, hi * static_cast<int>(wc));
+                    }
+                    if (lane == i) {
+                        m0 = a0;
+                        m1 = a1;
+                        m2 = a2;
+                    }
+                }
+                const int sc = seg * 32 + lane;
+                if (m1)
+                    atomicAdd(s_acc + sc, static_cast<unsigned long long>(m1));
+                if (m2)
+                    atomicAdd(s_acc + kScans + sc, static_cast<unsigned long long>(m2));
+                if (m0)
+                    atomicAdd(s_acc + 2 * kScans + sc, static_cast<unsigned long long>(m0));
+            }
+            if (S.form == kPaired) {
+                if (over > (W == 1 ? 0xFFu : 0xFFFFu))
+                    report(st, kErrValue);
+                close_paired(S, st);
+            } else if (S.form == kSparse) {
+                int prev = -1;
+                bool bad = false;
+                for (uint32_t k = 0; k < S.c; ++k) {
+                    if (S.bt.n < 9)
+                        S.bt.refill();
+                    const int pos = static_cast<int>(S.bt.get(9));
+                    if (S.br.n < 16)
+                        S.br.refill();
+                    const long long val = S.br.get(8 * W);
+                    if (pos <= prev || val == 0) {
+                        bad = true;
+                        break;
+                    }
+                    prev = pos;
+                    atomicAdd(s_acc + pos, static_cast<unsigned long long>(val * wr));
+                    atomicAdd(s_acc + kScans + pos, static_cast<unsigned long long>(val * wc));
+                    atomicAdd(s_acc + 2 * kScans + pos, static_cast<unsigned long long>(val));
+                }
+                if (bad) {
+                    report(st, kErrSparse);
+                } else {
+                    const int pad = static_cast<int>(((9u * S.c + 7u) / 8u) * 8u - 9u * S.c);
+                    if (pad) {
+                        if (S.bt.n < pad)
+                            S.bt.refill();
+                        if (S.bt.get(pad) != 0u)
+                            report(st, kErrPad);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < 3 * kScans; i += blockDim.x) {
+            out[(static_cast<long long>(i / kScans) * rows + row) * kScans + (i % kScans)] =
+                static_cast<long long>(s_acc[i]);
+            s_acc[i] = 0ull;
+        }
+        __syncthreads();
+    }
+}
+
 template <int W>
 __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_t *__restrict__ dec_g,
                                                           long long first, long long nblk, void *__restrict__ out,
@@ -1580,17 +1751,43 @@ __global__ void k_amplitude(const T *__restrict__ in, float *__restrict__ out, l
         out[i] = sqrtf(static_cast<float>(in[i]));
 }
 
+// SM count of the current device (cached per device).
 int sm_count()
 {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0)
-            n = 1;
-    }
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end())
+        return it->second;
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0)
+        n = 1;
+    cache[dev] = n;
     return n;
+}
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device (the attribute belongs to each device's context), once.
+cudaError_t ensure_smem(const void *fn, size_t bytes)
+{
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lk(mu);
+    size_t &have = done[std::make_pair(fn, dev)];
+    if (have >= bytes)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e == cudaSuccess)
+        have = bytes;
+    return e;
 }
 
 constexpr size_t kTableBytes = static_cast<size_t>(kModels) * kStates * sizeof(uint32_t);
@@ -1893,15 +2090,10 @@ cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const
 {
     const dim3 grid((P + kCompactThreads - 1) / kCompactThreads, nblk);
     const int smem = kCompactBytes + 32;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(k_enc_compact<uint8_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(k_enc_compact<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-        attr = true;
-    }
+    cudaError_t e = w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_enc_compact<uint8_t>), smem)
+                           : ensure_smem(reinterpret_cast<const void *>(k_enc_compact<uint16_t>), smem);
+    if (e != cudaSuccess)
+        return e;
     if (w == 1)
         k_enc_compact<uint8_t><<<grid, kCompactThreads, smem, st>>>(static_cast<const uint8_t *>(counts), P, nblk,
                                                                      desc, slots, blk_dst);
@@ -1935,14 +2127,9 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
     const size_t smem = kTableBytes +
                         static_cast<size_t>(TH / 32) * 16 * sizeof(uint32_t) +
                         static_cast<size_t>(kMaxSlots) * kScans * sizeof(uint32_t);
-    static size_t attr = 0;
-    if (attr < smem) {
-        const cudaError_t e = cudaFuncSetAttribute(k_decode_reduce<W, TH, DELTA>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess)
-            return e;
-        attr = smem;
-    }
+    const cudaError_t e = ensure_smem(reinterpret_cast<const void *>(k_decode_reduce<W, TH, DELTA>), smem);
+    if (e != cudaSuccess)
+        return e;
     // programmatic dependent launch: the CTAs may become resident and load their
     // tables while the preceding kernel (the plan) is still running
     cudaLaunchConfig_t cfg = {};
@@ -1963,8 +2150,10 @@ cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const 
                                  long long rows, void *out, int out_bytes, DevStatus *status, int n_sm,
                                  cudaStream_t st, bool delta, void *keep, IndexView ix)
 {
+    // u8 deltas (few tasks, each warp's decode latency is the critical path)
+    // run at 512 threads, with room for more registers; full queries at 768
     if (v.w == 1)
-        return delta ? launch_dr<1, 768, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
+        return delta ? launch_dr<1, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
                                                n_sm, st)
                      : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
                                                 n_sm, st);
@@ -1979,23 +2168,33 @@ cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n
 {
     const size_t smem = kTableBytes;
     const int grid = sm_count();
-    if (v.w == 1) {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(k_decode_blocks<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-            attr = true;
-        }
+    const cudaError_t e = v.w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_decode_blocks<1>), smem)
+                                   : ensure_smem(reinterpret_cast<const void *>(k_decode_blocks<2>), smem);
+    if (e != cudaSuccess)
+        return e;
+    if (v.w == 1)
         k_decode_blocks<1><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
-    } else {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(k_decode_blocks<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-            attr = true;
-        }
+    else
         k_decode_blocks<2><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
-    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moments(View v, Tables tb, const uint32_t *list, const uint32_t *count, const int32_t *weights,
+                           int stride, long long rows, long long *out, DevStatus *status, cudaStream_t st)
+{
+    const size_t smem = kTableBytes + 3 * kScans * sizeof(unsigned long long);
+    const cudaError_t e = v.w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_moments<1>), smem)
+                                   : ensure_smem(reinterpret_cast<const void *>(k_moments<2>), smem);
+    if (e != cudaSuccess)
+        return e;
+    long long grid = rows < 1 ? 1 : rows;
+    grid = grid > sm_count() ? sm_count() : grid;
+    if (v.w == 1)
+        k_moments<1><<<static_cast<int>(grid), 512, smem, st>>>(v, tb.dec, list, count, weights, stride, rows, out,
+                                                                 status);
+    else
+        k_moments<2><<<static_cast<int>(grid), 512, smem, st>>>(v, tb.dec, list, count, weights, stride, rows, out,
+                                                                 status);
     return cudaGetLastError();
 }
 
@@ -2015,19 +2214,10 @@ cudaError_t launch_index_sums(View v, Tables tb, const uint32_t *slots, int L, l
 {
     const int skip_count = __builtin_popcount(tb.skip_models);
     const size_t smem = kTableBytes + 24 * 16 * sizeof(uint32_t);
-    static int attr_dev[2] = {-1, -1};
-    const int wi = v.w == 1 ? 0 : 1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (attr_dev[wi] != dev) {
-        const cudaError_t e = v.w == 1 ? cudaFuncSetAttribute(k_index_sums<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                              static_cast<int>(smem))
-                                       : cudaFuncSetAttribute(k_index_sums<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                              static_cast<int>(smem));
-        if (e != cudaSuccess)
-            return e;
-        attr_dev[wi] = dev;
-    }
+    const cudaError_t e = v.w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_index_sums<1>), smem)
+                                   : ensure_smem(reinterpret_cast<const void *>(k_index_sums<2>), smem);
+    if (e != cudaSuccess)
+        return e;
     if (v.w == 1)
         k_index_sums<1><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, slots, L, b0, nblk,
                                                   leafsum, status);

@@ -148,6 +148,9 @@ cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const 
                                  DevStatus *status, int n_sm, cudaStream_t st, bool delta = false,
                                  void *keep = nullptr, IndexView ix = IndexView{nullptr, nullptr, nullptr, 0, 0});
 cudaError_t launch_amplitude(const void *counts, int w, float *amp, long long n, cudaStream_t st);
+// masked moments: out int64 [3][rows][512] = (sum x*wr, sum x*wc, sum x) per scan
+cudaError_t launch_moments(View v, Tables tb, const uint32_t *list, const uint32_t *count, const int32_t *weights,
+                           int stride, long long rows, long long *out, DevStatus *status, cudaStream_t st);
 // interaction index build (leafsum zeroed by the caller: [nblk][L][512] u32)
 cudaError_t launch_index_sums(View v, Tables tb, const uint32_t *slots, int L, long long b0, int nblk,
                               uint32_t *leafsum, DevStatus *status, int n_sm, cudaStream_t st);
