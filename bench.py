@@ -324,6 +324,10 @@ def run_profile_case(dev, torch, V):
     for t, d in enumerate(w.drag[:6]):
         md = torch.from_numpy(d).to(dev)
         (res.masked_sum_delta if t else res.masked_sum)(md, out=out)
+    # the schedule's other strides (launches 10..13: bf k4, adf k4, bf k16, adf k16)
+    for k in (4, 16):
+        for m in (bf, adf):
+            res.masked_sum(m, block_stride=k, out=out[: -(-w.n_blocks // k)])
     p = res.profile_read()
     print(json.dumps({"encode_s": t_enc, "kernels": p}), flush=True)
     res.free()
@@ -585,6 +589,19 @@ def main():
         d["enc_gbs"] = d["enc_bytes"] / (d["ms"] / 1e3) / 1e9
 
     hbm, peak_kind = peaks()
+    # DRAM traffic per decode launch from a committed ncu capture, if it was taken on
+    # this exact kernel source (else null)
+    traffic = None
+    try:
+        import hashlib
+        with open(os.path.join(ROOT, "virtual_imaging_b200", "csrc", "kernels.cu"), "rb") as f:
+            src_hash = hashlib.sha256(f.read()).hexdigest()
+        with open(os.path.join(ROOT, "profiles", "k_decode_reduce_c4_traffic.json")) as f:
+            tj = json.load(f)
+        if args.config == "c4" and tj.get("kernels_cu_sha256") == src_hash:
+            traffic = tj["schedule_bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        traffic = None
     n_dec, ms_dec = prof["decode_reduce"]
     bytes_step = sum(a["bytes"] for a in ab)
     raw_step = sum(a["raw"] for a in ab)
@@ -609,7 +626,7 @@ def main():
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": (achieved / hbm) if achieved else None, "traffic": None,
+                     "frac": (achieved / hbm) if achieved else None, "traffic": traffic,
                      "kernel": "k_decode_reduce", "peak_kind": peak_kind,
                      "avg_launch_ms": ms_dec / max(1, n_dec), "launches": n_dec,
                      "algorithmic_bytes_per_launch": bytes_step * args.steps / max(1, n_dec)},

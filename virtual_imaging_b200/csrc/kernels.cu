@@ -1490,11 +1490,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
 // through warp reductions of 32-bit partial sums (for 16-bit counts the value
 // is split in bytes, so every partial sum stays below 2^31 for |w| < 2^18);
 // sparse streams scatter their nonzeros into the row with shared atomics.
-// Paired streams of every model use the general decode (decode tables of all
-// 32 models in shared memory).
+// Low-dose paired streams are decoded by run events (the run tables of those
+// models in shared memory, as in the masked sum) and scatter their nonzero
+// counts; other paired streams use the general decode.
 template <int W>
 __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__restrict__ dec_g,
-                                                   const uint32_t *__restrict__ list,
+                                                   const uint32_t *__restrict__ runs_g, uint32_t skip_models,
+                                                   int skip_count, const uint32_t *__restrict__ list,
                                                    const uint32_t *__restrict__ count,
                                                    const int32_t *__restrict__ weights, int stride, long long rows,
                                                    long long *__restrict__ out, DevStatus *__restrict__ st)
@@ -1503,8 +1505,11 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
     uint32_t *s_dec = smem;
     unsigned long long *s_acc = reinterpret_cast<unsigned long long *>(smem + kModels * kStates);  // [3][512]
     __shared__ unsigned s_next;
+    // the run-event tables of the low-dose models, then the other decode tables
     for (int i = threadIdx.x; i < kModels * kStates / 4; i += blockDim.x)
-        reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
+        reinterpret_cast<uint4 *>(s_dec)[i] = i < skip_count * kStates / 4
+                                                  ? __ldg(reinterpret_cast<const uint4 *>(runs_g) + i)
+                                                  : __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
     for (int i = threadIdx.x; i < 3 * kScans; i += blockDim.x)
         s_acc[i] = 0ull;
     const uint32_t n = __ldg(count), n_l = __ldg(count + 1);
@@ -1550,13 +1555,16 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
                 ok = open_stream(S, W, st);
             if (!ok)
                 S.form = kEmpty;
-            const bool dense_lane = S.form == kPaired || S.form == kLiteral || S.form == kConstant;
+            // low-dose paired streams: run events scattered after the dense loop
+            const bool run_model = (skip_models >> S.model) & 1u;
+            const bool runs = S.form == kPaired && S.shift == 0 && S.base == 0u && run_model;
+            const bool dense_lane = (S.form == kPaired && !runs) || S.form == kLiteral || S.form == kConstant;
             const bool dense = __any_sync(kFull, dense_lane);
-            const uint32_t *dec = s_dec + S.model * kStates;
+            const uint32_t *dec = (run_model ? dec_g : s_dec) + S.model * kStates;
             uint32_t over = 0;
             for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
                 uint32_t vv[32];
-                if (S.form == kPaired) {
+                if (S.form == kPaired && !runs) {
                     paired_segment(S, dec, vv, over);
                 } else if (S.form == kLiteral) {
 #pragma unroll
@@ -1601,7 +1609,41 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
                 if (m0)
                     atomicAdd(s_acc + 2 * kScans + sc, static_cast<unsigned long long>(m0));
             }
-            if (S.form == kPaired) {
+            if (runs) {
+                // one event per iteration (see decode_task): jump the zero-bit run,
+                // then the landing slot's step; its nonzero counts scatter
+                const uint32_t *rt = s_dec + S.model * kStates;
+                int j = 0;
+                bool bad = false;
+                while (j < kPairs) {
+                    const uint32_t t = rt[S.x];
+                    j += static_cast<int>((t >> 14) & 63u);
+                    if (j >= kPairs) {
+                        bad = j > kPairs;
+                        S.x = (t >> 28) & 1u;
+                        break;
+                    }
+                    if (S.bt.n < 10)
+                        S.bt.refill();
+                    S.x = (t & 1023u) | S.bt.get(static_cast<int>((t >> 10) & 15u));
+                    const long long a = (t >> 20) & 15u, c = (t >> 24) & 15u;
+                    if (a) {
+                        atomicAdd(s_acc + 2 * j, static_cast<unsigned long long>(a * wr));
+                        atomicAdd(s_acc + kScans + 2 * j, static_cast<unsigned long long>(a * wc));
+                        atomicAdd(s_acc + 2 * kScans + 2 * j, static_cast<unsigned long long>(a));
+                    }
+                    if (c) {
+                        atomicAdd(s_acc + 2 * j + 1, static_cast<unsigned long long>(c * wr));
+                        atomicAdd(s_acc + kScans + 2 * j + 1, static_cast<unsigned long long>(c * wc));
+                        atomicAdd(s_acc + 2 * kScans + 2 * j + 1, static_cast<unsigned long long>(c));
+                    }
+                    ++j;
+                }
+                if (bad)
+                    report(st, kErrState);
+                else
+                    close_paired(S, st);
+            } else if (S.form == kPaired) {
                 if (over > (W == 1 ? 0xFFu : 0xFFFFu))
                     report(st, kErrValue);
                 close_paired(S, st);
@@ -2183,6 +2225,7 @@ cudaError_t launch_moments(View v, Tables tb, const uint32_t *list, const uint32
                            int stride, long long rows, long long *out, DevStatus *status, cudaStream_t st)
 {
     const size_t smem = kTableBytes + 3 * kScans * sizeof(unsigned long long);
+    const int skip_count = __builtin_popcount(tb.skip_models);
     const cudaError_t e = v.w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_moments<1>), smem)
                                    : ensure_smem(reinterpret_cast<const void *>(k_moments<2>), smem);
     if (e != cudaSuccess)
@@ -2190,11 +2233,11 @@ cudaError_t launch_moments(View v, Tables tb, const uint32_t *list, const uint32
     long long grid = rows < 1 ? 1 : rows;
     grid = grid > sm_count() ? sm_count() : grid;
     if (v.w == 1)
-        k_moments<1><<<static_cast<int>(grid), 512, smem, st>>>(v, tb.dec, list, count, weights, stride, rows, out,
-                                                                 status);
+        k_moments<1><<<static_cast<int>(grid), 512, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, list,
+                                                                 count, weights, stride, rows, out, status);
     else
-        k_moments<2><<<static_cast<int>(grid), 512, smem, st>>>(v, tb.dec, list, count, weights, stride, rows, out,
-                                                                 status);
+        k_moments<2><<<static_cast<int>(grid), 512, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, list,
+                                                                 count, weights, stride, rows, out, status);
     return cudaGetLastError();
 }
 
