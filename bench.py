@@ -472,45 +472,52 @@ def main():
     prof = res.profile_read()
     res.profile(False)
 
-    # end to end: masks from pinned host memory in, images to pinned host memory out
-    host_masks = [torch.from_numpy(m.astype(np.uint8)).pin_memory() for (_, m, _, _) in sched]
-    dev_masks = [torch.empty_like(h, device=dev) for h in host_masks]
-    host_imgs = [torch.empty(tuple(outs[k].shape), dtype=outs[k].dtype).pin_memory() for (_, _, k, _) in sched]
-    h2d = sum(h.numel() for h in host_masks)
-    d2h = sum(h.numel() * h.element_size() for h in host_imgs)
-
-    # Copies run on their own stream so that each image is read back while the
-    # next queries compute: masks go up on the copy stream and the query waits
-    # for them; an image goes down once its query is done; each stride has two
-    # output buffers used in turn, and a query waits until the read-back of the
-    # buffer it is about to overwrite has finished.
+    # end to end: each step's masks go up from pinned host memory in one copy, every
+    # query writes its own image, and the step's images come back to pinned host
+    # memory in one copy on a second stream, overlapping the next step's queries.
+    # Two sets of device buffers are used in turn; a step waits until the read-back
+    # of the set it is about to overwrite has finished.
+    P = w.n_pixels
+    nq_ = len(sched)
+    host_masks = torch.from_numpy(np.stack([m.astype(np.uint8) for (_, m, _, _) in sched])).pin_memory()
+    img_elems = [(-(-w.n_blocks // k)) * 512 for (_, _, k, _) in sched]
+    img_off = np.concatenate([[0], np.cumsum(img_elems)])
+    odt = V.out_dtype(out_bits)
+    sets = []
+    for _ in range(2):
+        dmask = torch.empty((nq_, P), dtype=torch.uint8, device=dev)
+        dimg = torch.empty(int(img_off[-1]), dtype=odt, device=dev)
+        himg = torch.empty(int(img_off[-1]), dtype=odt).pin_memory()
+        views = [dimg[int(img_off[i]):int(img_off[i + 1])].view(-1, 512) for i in range(nq_)]
+        sets.append({"mask": dmask, "img": dimg, "host": himg, "views": views, "free": None})
+    h2d = host_masks.numel()
+    d2h = int(img_off[-1]) * sets[0]["img"].element_size()
     comp_st = torch.cuda.current_stream(dev)
     copy_st = torch.cuda.Stream(device=dev)
-    bufs = {k: [outs[k], torch.empty_like(outs[k])] for k in outs}
-    turn = {k: 0 for k in outs}
-    freed = {k: [None, None] for k in outs}
+    turn = [0]
 
     def e2e_step():
-        for (label, m, k, delta), hm, dm, hi in zip(sched, host_masks, dev_masks, host_imgs):
-            with torch.cuda.stream(copy_st):
-                dm.copy_(hm, non_blocking=True)
-            up = torch.cuda.Event()
-            up.record(copy_st)
-            comp_st.wait_event(up)
-            i = turn[k]
-            turn[k] ^= 1
-            if freed[k][i] is not None:
-                comp_st.wait_event(freed[k][i])
+        S = sets[turn[0]]
+        turn[0] ^= 1
+        if S["free"] is not None:
+            copy_st.wait_event(S["free"])
+            comp_st.wait_event(S["free"])
+        with torch.cuda.stream(copy_st):
+            S["mask"].copy_(host_masks, non_blocking=True)
+        up = torch.cuda.Event()
+        up.record(copy_st)
+        comp_st.wait_event(up)
+        for i, (label, m, k, delta) in enumerate(sched):
             fn = res.masked_sum_delta if delta else res.masked_sum
-            fn(dm, block_stride=k, out=bufs[k][i], wait=False, stream=comp_st)
-            done = torch.cuda.Event()
-            done.record(comp_st)
-            copy_st.wait_event(done)
-            with torch.cuda.stream(copy_st):
-                hi.copy_(bufs[k][i], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(copy_st)
-            freed[k][i] = ev
+            fn(S["mask"][i], block_stride=k, out=S["views"][i], wait=False, stream=comp_st)
+        done = torch.cuda.Event()
+        done.record(comp_st)
+        copy_st.wait_event(done)
+        with torch.cuda.stream(copy_st):
+            S["host"].copy_(S["img"], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(copy_st)
+        S["free"] = ev
 
     e2e_step()
     res.finish()
@@ -527,6 +534,13 @@ def main():
     res.finish()
     te = f0.elapsed_time(f1) / 1e3
     te = max_over_ranks(te, device=dev)
+    # the read-back images are the queries' results: the last step's first image
+    # against a fresh query of the same mask
+    last = sets[turn[0] ^ 1]
+    lbl0, m0_, k0_, _ = sched[0]
+    ref0 = res.masked_sum(torch.from_numpy(m0_.astype(np.uint8)).to(dev), block_stride=k0_,
+                          out_bits=out_bits).cpu()
+    e2e_exact = bool(torch.equal(last["host"][: int(img_off[1])].view(-1, 512), ref0))
 
     # fused moments (centre-of-mass numerators and denominator) over the bright-field
     # disk and the annulus, stride 1: every masked pixel decoded, 10 back to back
@@ -623,7 +637,7 @@ def main():
                    "resident_bytes": info["payload_bytes"] + info["group_bytes"], "raw_bytes": w.raw_bytes},
         "raw_equiv_gbs": world * raw_step * args.steps / t / 1e9,
         "e2e": {"value": world * nq * args.steps / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h), "images_checked": e2e_exact},
         "gpu_launches": int(launches),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": (achieved / hbm) if achieved else None, "traffic": traffic,
