@@ -178,6 +178,15 @@ int qem_build_index(qem_resident *res, double center_row, double center_col, voi
  * Synchronises `stream` first. */
 int qem_drop_index(qem_resident *res, void *stream);
 
+/* The polar layout qem_build_index would use for this geometry, computed on
+ * the host only (no device work): arguments and outputs as for
+ * qem_index_layout; h_valid (host, n_pixels bytes, may be NULL = all valid).
+ * Call once with h_slots and h_root_leaf0 NULL to learn the sizes.
+ * QEM_ERR_ARG for an empty or too large detector or a non-finite centre. */
+int qem_polar_layout(int32_t det_rows, int32_t det_cols, const uint8_t *h_valid, double center_row,
+                     double center_col, uint32_t *h_slots, int32_t *h_root_leaf0, int32_t *n_leaves,
+                     int32_t *n_roots);
+
 /* The index's polar layout, for inspection: *n_leaves and *n_roots (may be
  * NULL); h_slots (host, may be NULL) receives 64 pixel indices per leaf, in
  * leaf order, with n_pixels marking unused slots of a sector's last leaf;

@@ -32,7 +32,7 @@ EXPORTS = ("qem_abi", "qem_status_string", "qem_create", "qem_encode", "qem_enco
            "qem_profile", "qem_profile_read", "qem_free", "qem_block_bytes", "qem_export_block", "qem_import",
            "qem_model_tables", "qem_generate_counts", "qem_masked_sum_noalloc", "qem_build_index",
            "qem_drop_index", "qem_index_layout", "qem_index_desc", "qem_export_valid", "qem_save", "qem_load",
-           "qem_decode_blocks_amplitude", "qem_masked_moments")
+           "qem_decode_blocks_amplitude", "qem_masked_moments", "qem_polar_layout")
 
 
 class QemError(RuntimeError):
@@ -108,6 +108,8 @@ def lib() -> ctypes.CDLL:
         "qem_load": ([ctypes.c_char_p, vp, pp], ctypes.c_int),
         "qem_decode_blocks_amplitude": ([vp, i64, i64, vp, vp, i32, vp], ctypes.c_int),
         "qem_masked_moments": ([vp, vp, vp, i32, vp, i32, vp], ctypes.c_int),
+        "qem_polar_layout": ([i32, i32, vp, ctypes.c_double, ctypes.c_double, vp, vp, ctypes.POINTER(i32),
+                              ctypes.POINTER(i32)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -136,8 +138,11 @@ def _check(code: int, where: str):
 
 
 def _stream(stream=None) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream
+    if stream is None:
+        if not torch.cuda.is_available():
+            return 0        # the default stream; calls that need a device then fail in the library
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
 
 
 def _dev_ptr(t: torch.Tensor | None) -> int:
@@ -381,6 +386,21 @@ class Resident:
             self.free()
         except Exception:
             pass
+
+
+def polar_layout(det_rows: int, det_cols: int, center, valid: np.ndarray | None = None):
+    """Host-only: (slots int64 [leaves][64], root_leaf0 int64 [roots + 1]) of the index layout."""
+    v = None if valid is None else np.ascontiguousarray(valid, np.uint8)
+    nl, nr = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().qem_polar_layout(det_rows, det_cols, None if v is None else v.ctypes.data, float(center[0]),
+                                  float(center[1]), None, None, ctypes.byref(nl), ctypes.byref(nr)),
+           "qem_polar_layout")
+    slots = np.zeros((nl.value, 64), np.uint32)
+    roots = np.zeros(nr.value + 1, np.int32)
+    _check(lib().qem_polar_layout(det_rows, det_cols, None if v is None else v.ctypes.data, float(center[0]),
+                                  float(center[1]), slots.ctypes.data, roots.ctypes.data, None, None),
+           "qem_polar_layout")
+    return slots.astype(np.int64), roots.astype(np.int64)
 
 
 def model_tables():

@@ -1091,6 +1091,29 @@ int qem_drop_index(qem_resident *r, void *stream)
     return QEM_OK;
 }
 
+int qem_polar_layout(int32_t det_rows, int32_t det_cols, const uint8_t *h_valid, double center_row,
+                     double center_col, uint32_t *h_slots, int32_t *h_root_leaf0, int32_t *n_leaves,
+                     int32_t *n_roots)
+{
+    if (det_rows <= 0 || det_cols <= 0 || !std::isfinite(center_row) || !std::isfinite(center_col) ||
+        static_cast<int64_t>(det_rows) * det_cols > (int64_t(1) << 24) - 1)
+        return QEM_ERR_ARG;
+    std::vector<uint8_t> valid(static_cast<size_t>(det_rows) * det_cols, 1);
+    if (h_valid)
+        for (size_t i = 0; i < valid.size(); ++i)
+            valid[i] = h_valid[i] ? 1 : 0;
+    const PolarLayout lay = polar_layout(det_rows, det_cols, valid, center_row, center_col);
+    if (n_leaves)
+        *n_leaves = lay.L;
+    if (n_roots)
+        *n_roots = lay.R;
+    if (h_slots)
+        std::memcpy(h_slots, lay.slots.data(), lay.slots.size() * 4);
+    if (h_root_leaf0)
+        std::memcpy(h_root_leaf0, lay.root_leaf0.data(), lay.root_leaf0.size() * 4);
+    return QEM_OK;
+}
+
 int qem_index_layout(const qem_resident *r, uint32_t *h_slots, int32_t *h_root_leaf0, int32_t *n_leaves,
                      int32_t *n_roots)
 {
