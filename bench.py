@@ -630,8 +630,11 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u8" if w.dtype_bits == 8 else "u16", "data": "synthetic",
         "config": {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
-                               f"uint{w.dtype_bits}, counter-based Poisson (BF r=30 lambda=3, outside 0.01)",
-                   "queries_per_step": nq, "schedule": "bf/adf at block_stride 1,4,16 + drag: 1 full + 64 deltas",
+                               f"uint{w.dtype_bits}, counter-based Poisson"
+                               + (" (BF r=30 lambda=3, outside 0.01)" if w.name == "c4" else ""),
+                   "queries_per_step": nq,
+                   "schedule": "bf/adf at block_stride " + ",".join(str(k) for k in w.strides)
+                               + (f" + drag: 1 full + {len(w.drag) - 1} deltas" if w.drag else ""),
                    "parallelism": f"{world} independent residents (one per GPU)",
                    "l2": f"inputs larger than L2: {bytes_step / 1e9:.2f} GB of encoded streams read per step",
                    "resident_bytes": info["payload_bytes"] + info["group_bytes"], "raw_bytes": w.raw_bytes},
