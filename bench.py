@@ -474,9 +474,11 @@ def main():
 
     # end to end: each step's masks go up from pinned host memory in one copy, every
     # query writes its own image, and the step's images come back to pinned host
-    # memory in one copy on a second stream, overlapping the next step's queries.
-    # Two sets of device buffers are used in turn; a step waits until the read-back
-    # of the set it is about to overwrite has finished.
+    # memory in one copy, overlapping the next step's queries.  Uploads and
+    # read-backs run on two copy streams of their own (opposite directions), so the
+    # next step's upload does not queue behind this step's read-back.  Two sets of
+    # device buffers are used in turn; a step waits until the read-back of the set
+    # it is about to overwrite has finished.
     P = w.n_pixels
     nq_ = len(sched)
     host_masks = torch.from_numpy(np.stack([m.astype(np.uint8) for (_, m, _, _) in sched])).pin_memory()
@@ -493,30 +495,33 @@ def main():
     h2d = host_masks.numel()
     d2h = int(img_off[-1]) * sets[0]["img"].element_size()
     comp_st = torch.cuda.current_stream(dev)
-    copy_st = torch.cuda.Stream(device=dev)
+    up_st = torch.cuda.Stream(device=dev)
+    down_st = torch.cuda.Stream(device=dev)
     turn = [0]
 
     def e2e_step():
         S = sets[turn[0]]
         turn[0] ^= 1
         if S["free"] is not None:
-            copy_st.wait_event(S["free"])
+            # the read-back of this set two steps ago (which followed that step's
+            # queries, the last readers of its masks) has finished
+            up_st.wait_event(S["free"])
             comp_st.wait_event(S["free"])
-        with torch.cuda.stream(copy_st):
+        with torch.cuda.stream(up_st):
             S["mask"].copy_(host_masks, non_blocking=True)
         up = torch.cuda.Event()
-        up.record(copy_st)
+        up.record(up_st)
         comp_st.wait_event(up)
         for i, (label, m, k, delta) in enumerate(sched):
             fn = res.masked_sum_delta if delta else res.masked_sum
             fn(S["mask"][i], block_stride=k, out=S["views"][i], wait=False, stream=comp_st)
         done = torch.cuda.Event()
         done.record(comp_st)
-        copy_st.wait_event(done)
-        with torch.cuda.stream(copy_st):
+        down_st.wait_event(done)
+        with torch.cuda.stream(down_st):
             S["host"].copy_(S["img"], non_blocking=True)
         ev = torch.cuda.Event()
-        ev.record(copy_st)
+        ev.record(down_st)
         S["free"] = ev
 
     e2e_step()
@@ -528,7 +533,7 @@ def main():
     f0.record()
     for _ in range(args.steps):
         e2e_step()
-    comp_st.wait_stream(copy_st)
+    comp_st.wait_stream(down_st)
     f1.record()
     torch.cuda.synchronize()
     res.finish()
