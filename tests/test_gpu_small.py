@@ -19,7 +19,7 @@ from qem_testlib import export_all, gpu_encode, image, oracle_resident, to_dev
 
 pytestmark = pytest.mark.gpu
 
-SMALL = ["c1", "c2", "s17", "s19", "s257"]
+SMALL = ["c1", "c2", "s17", "s19", "s257", "u19"]
 
 
 @pytest.fixture(scope="module")
@@ -78,8 +78,9 @@ def test_decode_blocks_roundtrip(data, name):
     res.free()
 
 
-def test_delta_chain_c2(data):
-    w, x, enc = data("c2")
+@pytest.mark.parametrize("name", ["c2", "u19"])
+def test_delta_chain(data, name):
+    w, x, enc = data(name)
     res = gpu_encode(w, x)
     for k in (1, 3):
         img = image(res, w.drag[0], k)

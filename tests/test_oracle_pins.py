@@ -290,7 +290,30 @@ def test_group_layout_invariants():
 # ----------------------------------------------------------------------------
 # queries against brute force
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("name", ["c1", "c2", "s17", "s19"])
+def test_u8_mixed_fixture_mixes_stream_kinds():
+    """The uint8 fixture for mixed warps: every block has 32-pixel groups holding
+    plain paired streams beside paired streams with raw low bits (shift > 0),
+    and low-dose run-model streams as well."""
+    w = W.workload("u19")
+    enc = O.encode(w.host_counts(), 8)
+    for b in range(w.n_blocks):
+        g, pay = enc.groups[b], enc.payloads[b]
+        mixed = runs = 0
+        for gi in range(g.shape[0]):
+            ends = [0] + [(int(g[gi, 1 + j // 2]) >> (16 * (j & 1))) & 0xFFFF for j in range(32)]
+            kinds = set()
+            for j in range(32):
+                a, e = int(g[gi, 0]) + ends[j], int(g[gi, 0]) + ends[j + 1]
+                if e > a:
+                    h = int(pay[a]) | (int(pay[a + 1]) << 8)
+                    if h & 7 == 3:
+                        kinds.add("shifted" if (h >> 8) & 15 else ("runs" if (h >> 3) & 31 < 8 else "plain"))
+            mixed += {"plain", "shifted"} <= kinds
+            runs += "runs" in kinds
+        assert mixed >= 5 and runs >= 5, (b, mixed, runs)
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "s17", "s19", "u19"])
 def test_masked_sum_equals_dense(name):
     w = W.workload(name)
     x = w.host_counts()

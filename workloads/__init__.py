@@ -275,6 +275,21 @@ def _small_counts(w: Workload) -> np.ndarray:
     return counts.astype(w.np_dtype)
 
 
+def _u8_mixed_counts(w: Workload) -> np.ndarray:
+    """uint8 fixture for warps mixing stream kinds: per-pixel Poisson means
+    in [0.3, 3.5] (streams of plain pair steps) and a fifth of the pixels at
+    0.01 (run events or sparse), and 48 planted counts in [16, 200] that give
+    their streams raw low bits (shift > 0) beside plain neighbours."""
+    rng = np.random.default_rng(w.seed)
+    lam = rng.uniform(0.3, 3.5, size=w.n_pixels)
+    lam[rng.random(w.n_pixels) < 0.2] = 0.01
+    counts = rng.poisson(np.broadcast_to(lam, (w.n_scans, w.n_pixels)))
+    s = rng.integers(0, w.n_scans, size=48)
+    p = rng.integers(0, w.n_pixels, size=48)
+    counts[s, p] = rng.integers(16, 201, size=48)
+    return np.minimum(counts, 255).astype(np.uint8)
+
+
 _HOST_GEN = {"c1": _c1_counts, "c2": _c2_counts}
 
 
@@ -352,6 +367,14 @@ def workload(name: str) -> Workload:
         w.masks = {"full": np.ones(det * det, dtype=np.uint8), "bf": disk(det, det, c, c, det // 4),
                    "adf": annulus(det, det, c, c, det // 4 + 1, det // 2)}
         _HOST_GEN[name] = _small_counts
+        return w
+    if name == "u19":
+        det, c = 19, 9
+        w = Workload(name, 32, 32, det, det, 8, 19, "host")
+        w.masks = {"full": np.ones(det * det, dtype=np.uint8), "bf": disk(det, det, c, c, 4),
+                   "adf": annulus(det, det, c, c, 5, 9)}
+        w.drag = [disk(det, det, c, 4 + t, 4) for t in range(11)]
+        _HOST_GEN[name] = _u8_mixed_counts
         return w
     raise KeyError(name)
 
