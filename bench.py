@@ -248,6 +248,17 @@ def cpu_baseline(w, sample_blocks=4):
                       f"{n} queries in {dt * n:.1f} s, scaled to all blocks"}
 
 
+def workload_config(w, nq, world):
+    """The workload part of the bench line's config, the same for both arms."""
+    return {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
+                        f"uint{w.dtype_bits}, counter-based Poisson"
+                        + (" (BF r=30 lambda=3, outside 0.01)" if w.name == "c4" else ""),
+            "queries_per_step": nq,
+            "schedule": "bf/adf at block_stride " + ",".join(str(k) for k in w.strides)
+                        + (f" + drag: 1 full + {len(w.drag) - 1} deltas" if w.drag else ""),
+            "parallelism": f"{world} independent residents (one per GPU)"}
+
+
 def run_reference(args, rank, world):
     """The oracle timed on the host cores on a bounded sample (2 blocks) of the same workload and schedule:
     every query of the step runs over the sampled blocks, and its time per block is scaled by the number
@@ -287,8 +298,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_full * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u8" if w.dtype_bits == 8 else "u16",
             "data": "synthetic",
-            "config": {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
-                                   f"uint{w.dtype_bits}", "queries_per_step": len(sched)},
+            "config": workload_config(w, len(sched), world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"each of the {len(sched)} queries of a step timed over blocks {blocks} of "
                                        f"{w.n_blocks} and scaled to the ceil(B/k) blocks it touches"},
@@ -634,13 +644,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u8" if w.dtype_bits == 8 else "u16", "data": "synthetic",
-        "config": {"workload": f"{w.name}: scan {w.scan_rows}x{w.scan_cols}, detector {w.det_rows}x{w.det_cols}, "
-                               f"uint{w.dtype_bits}, counter-based Poisson"
-                               + (" (BF r=30 lambda=3, outside 0.01)" if w.name == "c4" else ""),
-                   "queries_per_step": nq,
-                   "schedule": "bf/adf at block_stride " + ",".join(str(k) for k in w.strides)
-                               + (f" + drag: 1 full + {len(w.drag) - 1} deltas" if w.drag else ""),
-                   "parallelism": f"{world} independent residents (one per GPU)",
+        "config": {**workload_config(w, nq, world),
                    "l2": f"inputs larger than L2: {bytes_step / 1e9:.2f} GB of encoded streams read per step",
                    "resident_bytes": info["payload_bytes"] + info["group_bytes"], "raw_bytes": w.raw_bytes},
         "raw_equiv_gbs": world * raw_step * args.steps / t / 1e9,
