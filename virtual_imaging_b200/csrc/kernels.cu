@@ -991,13 +991,15 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
 // ---------------------------------------------------------------------------
 // a6: fused decode + masked reduce (the hot kernel)
 // ---------------------------------------------------------------------------
-// Persistent CTAs, one per SM; the 32 models' decode tables (128 KB) live in
-// shared memory.  Work is a 1-D list of warp tasks (touched block row, tile of
-// 32 listed pixels); a CTA takes WARPS consecutive tasks at a time, each warp
-// decodes its 32 streams (one per lane) 32 scans at a time and reduces them
-// across the warp with redux.sync, adding each scan's total into a per-row
-// shared accumulator; the CTA then adds its rows to the output with one
-// global atomic per nonzero scan sum.
+// Persistent CTAs, one per SM; one 4 KB table per model (run-event tables of
+// the low-dose models, decode tables of the others) lives in shared memory.
+// Index items (whole pixel groups served from stored sums) go first.  Then the
+// decode work, a 1-D list of warp tasks (touched block row, tile of 32 listed
+// pixels), is cut into one contiguous share per CTA; its warps take tasks from
+// a shared counter.  Each warp decodes its 32 streams (one per lane) 32 scans
+// at a time and reduces them across the warp with redux.sync into the row's
+// shared slot; the warp that finishes a row piece's last task adds the slot to
+// the output with one global atomic per nonzero scan sum.
 template <int W, bool DELTA>
 __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint32_t *dec_g,
                                             uint32_t skip_models, const uint32_t *list, uint32_t n,
