@@ -10,11 +10,20 @@
 //    stream with a 64-bit bit reservoir refilled four bytes at a time once per
 //    three coded pairs, reduced warp-wide per 32 scans into exact integer
 //    virtual images, optionally over every k-th block only (k_decode_reduce);
-//  * step 6 -- whole blocks decode back to native patterns (k_decode_blocks).
+//  * step 3 -- the interaction index: exact per-scan sums of polar pixel
+//    groups, built by one decode pass (k_index_sums, k_index_size,
+//    k_index_pack); a full query takes the groups wholly inside its mask from
+//    them and decodes the rest (k_plan_index, index items in k_decode_reduce);
+//  * step 6 -- whole blocks decode back to native patterns (k_decode_blocks),
+//    optionally with their float32 square-root amplitude (k_amplitude).
+// Page "Backend Optimization Matrix", CoM/DPC rows: fused moment numerators
+// and denominator over the same decode (k_moments).
 // Bit-level choices follow the library's spec qem-pair-v1 (S1-S7).
 //
 // No kernel traps or asserts: malformed input sets flags in DevStatus and the
-// affected lane contributes zeros.  Every loop has a fixed trip count.
+// affected lane contributes zeros.  Every loop ends: a fixed trip count, a
+// position or counter that only advances, or a wait bounded by kWaitLimit
+// polls that sets kErrWait when it runs out.
 #include <cstdio>
 #include <type_traits>
 
@@ -897,16 +906,16 @@ __global__ void __launch_bounds__(kCompactThreads) k_enc_compact(const T *__rest
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 256;
 
-// Blocks [0, n_list_blocks) build the pixel list, one pixel per thread: a
-// warp ballots its 32 pixels and reserves room with one atomic per class.
+// Blocks [0, n_list_blocks) build the pixel list, one pixel per thread: each
+// warp ballots its 32 pixels and the block reserves room for all its warps
+// with one atomic per class.
 // Pixels of the heavy class (decoded pair by pair) fill the list from the
 // front (count[0]), light ones (empty, sparse, run-decoded) from the back
 // (count[1], list[P-1], list[P-2], ...), so that warps meet one kind of work.
 // Order inside a class does not matter to the sums (integer addition).
 // Full query: mask && valid; delta: pixels whose (mask && valid) changed
 // against the stored baseline mask, leaving pixels flagged in bit 31.  Every
-// thread then stores the new mask as the baseline.  A block reserves its
-// list slots with one atomic per class.  Blocks past n_list_blocks initialise
+// thread then stores the new mask as the baseline.  Blocks past n_list_blocks initialise
 // the rows: a full query zeroes the output and the kept image, a delta starts
 // the output from the kept image (the decode adds its terms to both).  The
 // counter pair of the next query (count_next) is cleared here, so that no
@@ -1480,9 +1489,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
 }
 
 // ---------------------------------------------------------------------------
-// a7: block decode into native frames
-// ---------------------------------------------------------------------------
-// ---------------------------------------------------------------------------
 // masked moments (fused CoM / DPC numerators and denominator)
 // ---------------------------------------------------------------------------
 // For every touched block row and scan: sum of x * wr[p], of x * wc[p] and of
@@ -1691,6 +1697,13 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
     }
 }
 
+// ---------------------------------------------------------------------------
+// a7: block decode into native frames
+// ---------------------------------------------------------------------------
+// One thread per stream of nblk blocks from `first`: the thread decodes its
+// stream's 512 counts in order and stores them down its pixel column of the
+// [n * 512][P] frames (neighbouring threads hold neighbouring pixels, so each
+// scan's stores are coalesced).  Invalid pixels come out 0.
 template <int W>
 __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_t *__restrict__ dec_g,
                                                           long long first, long long nblk, void *__restrict__ out,
