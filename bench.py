@@ -465,6 +465,12 @@ def main():
     for _ in range(args.warmup):
         step()
     res.finish()
+    # one more untimed step with the library's own counters: the streams its
+    # decode listed, to check the count behind the algorithmic bytes
+    res.counters()
+    step()
+    res.finish()
+    _, streams_kernel = res.counters()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -665,6 +671,8 @@ def main():
         "e2e": {"value": world * nq * args.steps / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "images_checked": e2e_exact},
         "gpu_launches": int(launches),
+        "accounting": {"streams_per_step_decoded": int(streams_kernel),
+                       "streams_per_step_counted": int(sum(a["streams"] for a in ab))},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": (achieved / hbm) if achieved else None, "traffic": traffic,
                      "kernel": "k_decode_reduce", "peak_kind": peak_kind,
