@@ -26,6 +26,8 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
+import threading
 import sys
 import time
 
@@ -141,29 +143,87 @@ def algorithmic_bytes(lens, w, sched, out_bits, idx=None):
 
 
 class Clocks:
-    """nvidia-smi sampler (every 200 ms) around the timed region."""
+    """SM clock and clock-event reasons sampled during the timed region: through NVML (the
+    library nvidia-smi reads) every 10 ms on a background thread, else by nvidia-smi every
+    200 ms into a temporary file.  Reading only: no setting of the GPU is changed."""
 
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+    def __init__(self, index: int, uuid: str | None = None, period: float = 0.010):
+        self.index, self.uuid, self.period = index, uuid, period
+        self.samples = []            # (sm MHz, max sm MHz, reason names)
+        self.source = None
+        self.proc = self.thread = None
+        self.path = os.path.join(tempfile.gettempdir(), f"qem_clocks_{os.getpid()}_{index}.csv")
+
+    def _start_nvml(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            h = None
+            if self.uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid if self.uuid.startswith("GPU-")
+                                                         else "GPU-" + self.uuid)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            get_reasons = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                           or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+
+            def sample():
+                bits = int(get_reasons(h))
+                return (float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)), mx,
+                        tuple(n for n, b in self.REASONS if bits & b))
+
+            sample()                 # fails here if the device cannot be read
+        except Exception:
+            pynvml.nvmlShutdown()
+            raise
+        self._nvml = pynvml
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(sample())
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        self.source = "nvml"
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                                         stderr=subprocess.DEVNULL)
+            self._start_nvml()
         except Exception:
-            self.proc = None
+            try:
+                self.f = open(self.path, "w")
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                             stderr=subprocess.DEVNULL)
+                self.source = "nvidia-smi"
+            except Exception:
+                self.proc = None
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -171,27 +231,27 @@ class Clocks:
             except Exception:
                 self.proc.kill()
             self.f.close()
+            names = [n for n, _ in self.REASONS]
+            for line in open(self.path):
+                r = [x.strip() for x in line.split(",")]
+                if len(r) < 9 or not r[1].replace(".", "").isdigit() or not r[2].replace(".", "").isdigit():
+                    continue
+                self.samples.append((float(r[1]), float(r[2]),
+                                     tuple(names[i] for i in range(4) if r[5 + i].lower() == "active")))
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
 
     def summary(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append(parts)
-            except Exception:
-                pass
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": self.source}
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples),
+                "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": sorted({n for x in self.samples for n in x[2]}),
+                "samples": len(self.samples), "source": self.source}
 
 
 def build_resident(w, dev, torch, V, stream=None):
@@ -479,7 +539,11 @@ def main():
     # between the plan and decode launches of every query and cost ~0.8 ms per
     # step, so they are taken in the second timed pass below)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with Clocks(local) as clk:
+    try:
+        dev_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        dev_uuid = None
+    with Clocks(local, dev_uuid) as clk:
         e0.record()
         for _ in range(args.steps):
             step()

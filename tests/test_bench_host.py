@@ -92,3 +92,59 @@ def test_kernel_source_hash_ignores_comments(tmp_path, monkeypatch):
     k.write_text(text.replace("kFull = 0xFFFFFFFFu", "kFull = 0xFFFFFFFEu", 1))
     assert "kFull = 0xFFFFFFFEu" in k.read_text()
     assert bench.kernel_source_hash() != h0
+
+
+def _fake_nvml(fail=False):
+    import types
+
+    fake = types.ModuleType("pynvml")
+    st = {"init": 0, "shutdown": 0, "i": 0}
+
+    def init():
+        if fail:
+            raise RuntimeError("no driver")
+        st["init"] += 1
+
+    def by_uuid(u):
+        assert u.startswith("GPU-")
+        return "h"
+
+    def clock(h, c):
+        st["i"] += 1
+        return (1965, 1965, 1800)[st["i"] % 3]
+
+    fake.NVML_CLOCK_SM = 1
+    fake.nvmlInit = init
+    fake.nvmlShutdown = lambda: st.__setitem__("shutdown", st["shutdown"] + 1)
+    fake.nvmlDeviceGetHandleByUUID = by_uuid
+    fake.nvmlDeviceGetHandleByIndex = lambda i: "h"
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4 if st["i"] % 2 else 0x1
+    return fake, st
+
+
+def test_clock_sampler_reads_nvml(monkeypatch):
+    import sys
+    import time
+
+    fake, st = _fake_nvml()
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.Clocks(0, "0000-1111", period=0.001) as c:
+        time.sleep(0.05)
+    s = c.summary()
+    assert s["source"] == "nvml" and s["samples"] >= 5
+    assert s["sm_max_mhz"] == 1965 and s["sm_mhz"] in (1800, 1965)
+    assert s["reasons"] == ["sw_power_cap"]            # idle (0x1) is not a reason that matters
+    assert st["init"] == 1 and st["shutdown"] == 1
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    import sys
+
+    fake, _ = _fake_nvml(fail=True)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.Clocks(0) as c:
+        pass
+    s = c.summary()
+    assert s["sm_mhz"] is None and s["reasons"]
