@@ -66,3 +66,24 @@ def test_library_is_sm100a():
     assert "arch=compute_100a,code=sm_100a" in log
     assert "-lineinfo" in log
     np.zeros(1)
+
+
+def test_plain_c_consumer(tmp_path):
+    """include/qem.h compiles as pedantic C99 and the host-only entry points answer
+    through it from a C program linked against libqem.so (no GPU, no Python between)."""
+    V = _lib()
+    import shutil
+
+    import pytest
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = str(tmp_path / "c_abi_host")
+    libdir = os.path.dirname(V.LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_host.c"),
+                        "-L", libdir, "-lqem", f"-Wl,-rpath,{libdir}", "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.stdout, r.stderr)
