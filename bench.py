@@ -303,9 +303,33 @@ def cpu_baseline(w, sample_blocks=4):
             break
     dt = (time.perf_counter() - t0) / n
     full = dt * w.n_blocks / len(blocks)
-    return {"value": 1.0 / full, "unit": UNIT, "cores": threads, "kind": "oracle",
+    # the same queries on one core, over one block
+    one = O.Encoded(w.n_pixels, w.dtype_bits)
+    one.groups.append(enc.groups[0])
+    one.payloads.append(enc.payloads[0])
+    t1 = time.perf_counter()
+    for name in ("bf", "adf"):
+        O.resident_masked_sum(one, w.masks[name], None, 1, threads=1)
+    single = (time.perf_counter() - t1) / 2 * w.n_blocks
+    return {"value": 1.0 / full, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu": cpu_model(),
+            "single_core_value": 1.0 / single,
             "sample": f"bf/adf k=1 queries over {len(blocks)} of {w.n_blocks} blocks (host-regenerated), "
-                      f"{n} queries in {dt * n:.1f} s, scaled to all blocks"}
+                      f"{n} queries in {dt * n:.1f} s, scaled to all blocks; single core: one bf and one adf "
+                      f"query over block {blocks[0]}, scaled the same way"}
+
+
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo where there is one)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or platform.machine()
 
 
 def kernel_source_hash():
@@ -376,7 +400,7 @@ def run_reference(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "u8" if w.dtype_bits == 8 else "u16",
             "data": "synthetic",
             "config": workload_config(w, len(sched), world),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu": cpu_model(),
                              "sample": f"each of the {len(sched)} queries of a step timed over blocks {blocks} of "
                                        f"{w.n_blocks} and scaled to the ceil(B/k) blocks it touches"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
