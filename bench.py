@@ -551,10 +551,13 @@ def main():
     res.finish()
     # one more untimed step with the library's own counters: the streams its
     # decode listed, to check the count behind the algorithmic bytes
-    res.counters()
-    step()
-    res.finish()
-    _, streams_kernel = res.counters()
+    try:
+        res.counters()
+        step()
+        res.finish()
+        streams_kernel = int(res.counters()[1])
+    except V.QemError:
+        streams_kernel = None
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -759,7 +762,7 @@ def main():
         "e2e": {"value": world * nq * args.steps / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "images_checked": e2e_exact},
         "gpu_launches": int(launches),
-        "accounting": {"streams_per_step_decoded": int(streams_kernel),
+        "accounting": {"streams_per_step_decoded": streams_kernel,
                        "streams_per_step_counted": int(sum(a["streams"] for a in ab))},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": (achieved / hbm) if achieved else None, "traffic": traffic,
