@@ -546,6 +546,14 @@ def main():
             fn = res.masked_sum_delta if delta else res.masked_sum
             fn(md, block_stride=k, out=outs[k], wait=False)
 
+    # the first query after the build, timed alone: the cold figure
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    c0.record()
+    res.masked_sum(masks[0], block_stride=sched[0][2], out=outs[sched[0][2]], wait=False)
+    c1.record()
+    torch.cuda.synchronize()
+    cold = (sched[0][0], c0.elapsed_time(c1))
     for _ in range(args.warmup):
         step()
     res.finish()
@@ -715,19 +723,25 @@ def main():
         gbytes = np.where(codes > 0, 512 << np.maximum(codes.astype(np.int64) - 1, 0), 0)
         idx = (slots, roots, gbytes)
     ab = algorithmic_bytes(lens, w, sched, out_bits, idx)
+    # per query: the median of 20 warm passes over the schedule, each query timed
+    # alone (events around the call, synchronised after it)
     per_query = {}
-    for (label, m, k, delta), md, a in zip(sched, masks, ab):
-        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        fn = res.masked_sum_delta if delta else res.masked_sum
-        q0.record()
-        fn(md, block_stride=k, out=outs[k], wait=False)
-        q1.record()
-        torch.cuda.synchronize()
-        d = per_query.setdefault(label, {"ms": [], "enc_bytes": a["enc"], "raw_bytes": a["raw"]})
-        d["ms"].append(q0.elapsed_time(q1))
+    for _ in range(20):
+        for (label, m, k, delta), md, a in zip(sched, masks, ab):
+            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fn = res.masked_sum_delta if delta else res.masked_sum
+            q0.record()
+            fn(md, block_stride=k, out=outs[k], wait=False)
+            q1.record()
+            torch.cuda.synchronize()
+            d = per_query.setdefault(label, {"ms": [], "enc_bytes": a["enc"], "raw_bytes": a["raw"]})
+            d["ms"].append(q0.elapsed_time(q1))
     res.finish()
-    for d in per_query.values():
+    for label, d in per_query.items():
+        d["runs"] = len(d["ms"])
         d["ms"] = statistics.median(d["ms"])
+        if label == cold[0]:
+            d["cold_ms"] = cold[1]
         d["raw_equiv_gbs"] = d["raw_bytes"] / (d["ms"] / 1e3) / 1e9
         d["enc_gbs"] = d["enc_bytes"] / (d["ms"] / 1e3) / 1e9
 
@@ -769,8 +783,9 @@ def main():
                      "kernel": "k_decode_reduce", "peak_kind": peak_kind,
                      "avg_launch_ms": ms_dec / max(1, n_dec), "launches": n_dec,
                      "algorithmic_bytes_per_launch": bytes_step * args.steps / max(1, n_dec)},
-        "queries": {k: {"ms": round(v["ms"], 4), "raw_equiv_gbs": round(v["raw_equiv_gbs"], 1),
-                        "enc_gbs": round(v["enc_gbs"], 1), "hbm_frac_enc": round(v["enc_gbs"] / hbm, 4)}
+        "queries": {k: {"ms": round(v["ms"], 4), "runs": v["runs"], "raw_equiv_gbs": round(v["raw_equiv_gbs"], 1),
+                        "enc_gbs": round(v["enc_gbs"], 1), "hbm_frac_enc": round(v["enc_gbs"] / hbm, 4),
+                        **({"cold_ms": round(v["cold_ms"], 4)} if "cold_ms" in v else {})}
                     for k, v in per_query.items()},
         "kernels_ms_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[0]},
         "profiled_pass_ms_per_step": t_prof * 1e3 / args.steps,
