@@ -7,6 +7,7 @@ import subprocess
 import numpy as np
 
 import oracle as O
+from golden_io import frozen_tables as _frozen_tables, tables_sha as _sha
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -51,13 +52,47 @@ def test_abi_string_and_status_names():
     assert V.status_string(99) == "unknown status"
 
 
-def test_library_model_tables_equal_oracle():
-    """Host-side tables of the library, computed independently, equal the oracle's."""
+def test_frozen_tables_file_is_whole():
+    """The golden file's tables hash to the digest it states, and have the shapes and
+    sums spec S4 fixes (32 models, 256 pair symbols summing to 1024 states)."""
+    digest, f, a, c = _frozen_tables()
+    assert f.shape == (32, 256) and a.shape == (32,) and c.shape == (32, 16)
+    assert (f.astype(np.int64).sum(axis=1) == 1024).all()
+    assert _sha(f, a, c) == digest
+
+
+def test_oracle_rebuild_hashes_to_frozen_tables():
+    """The oracle rebuilds the models from spec S4 in double precision on this host;
+    its result must hash to the frozen digest (a libm that moved one floor() fails here)."""
+    digest, *_ = _frozen_tables()
+    assert _sha(*O.models()) == digest
+
+
+def test_library_tables_equal_frozen_tables():
+    """The library's tables (compiled from its own frozen data) equal the golden file."""
     V = _lib()
+    digest, f0, a0, c0 = _frozen_tables()
     f, a, c = V.model_tables()
-    f2, a2, c2 = O.models()
-    assert (f == f2).all() and (a == a2).all() and (c == c2).all()
-    assert (f.sum(axis=1) == 1024).all()
+    assert (f == f0).all() and (a == a0).all() and (c == c0).all()
+    assert _sha(f, a, c) == digest
+
+
+def test_library_frozen_data_is_its_generator_output(tmp_path):
+    """model_tables.inc is what the library's generator writes on this host."""
+    import shutil
+
+    import pytest
+
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    csrc = os.path.join(ROOT, "virtual_imaging_b200", "csrc")
+    exe = str(tmp_path / "gen")
+    r = subprocess.run([cxx, "-O2", "-std=c++17", "-o", exe, os.path.join(csrc, "gen_model_tables.cpp")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=60).stdout
+    assert out == open(os.path.join(csrc, "model_tables.inc")).read()
 
 
 def test_library_is_sm100a():

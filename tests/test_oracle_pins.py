@@ -16,6 +16,7 @@ from scipy import stats
 
 import oracle as O
 import workloads as W
+from golden_io import frozen_tables
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 LAM = lambda m: 0.005 * (16.0 / 0.005) ** (m / 31.0)
@@ -53,32 +54,74 @@ def test_contract_constants():
     assert g.dtype.itemsize * 8 == int(c["group_base_bits"])
 
 
+def _golden_bytes(text):
+    """Hex bytes with XX*n (a repeated byte) and (XX YY ..)*n (a repeated group)."""
+    import re
+
+    out = bytearray()
+    for grp, reps, tok in re.findall(r"\(([0-9A-Fa-f ]+)\)\*(\d+)|(\S+)", text):
+        if grp:
+            out += bytes(int(t, 16) for t in grp.split()) * int(reps)
+        elif "*" in tok:
+            b, n = tok.split("*")
+            out += bytes([int(b, 16)]) * int(n)
+        else:
+            out.append(int(tok, 16))
+    return bytes(out)
+
+
+def _golden_values(spec, w):
+    v = np.zeros(512, np.uint16)
+    kind, *args = spec.split()
+    if kind == "zeros":
+        pass
+    elif kind == "const":
+        v[:] = int(args[0])
+    elif kind == "sparse":
+        for t in args:
+            pos, val = t.split(":")
+            v[int(pos)] = int(val)
+    elif kind == "affine":
+        v[:] = (int(args[0]) * np.arange(512) + int(args[1])) % (1 << (8 * w))
+    elif kind == "based":
+        base, shift, mod = int(args[0]), int(args[1]), int(args[2])
+        hi = np.zeros(512, np.int64)
+        hi[[int(t) for t in args[3].split(",")]] = 1
+        v[:] = base + ((hi << shift) | (np.arange(512) % mod))
+    else:
+        raise AssertionError(kind)
+    return v
+
+
 def test_golden_forms():
+    """Hand-derived byte images of every form (tests/golden/forms.txt, derivations in
+    its comments): encode gives the bytes and decode gives the values back; dec_* rows
+    are decoder-only images (raw low bits beside the tANS section)."""
+    seen = set()
     for line in open(os.path.join(GOLDEN, "forms.txt")):
         if line.startswith("#") or not line.strip():
             continue
         name, w, spec, expected = (t.strip() for t in line.split("|"))
         w = int(w)
-        v = np.zeros(512, np.uint16)
-        kind, *args = spec.split()
-        if kind == "const":
-            v[:] = int(args[0])
-        elif kind == "sparse":
-            for t in args:
-                pos, val = t.split(":")
-                v[int(pos)] = int(val)
-        elif kind == "affine":
-            v[:] = (int(args[0]) * np.arange(512) + int(args[1])) % (1 << (8 * w))
-        got = O.encode_stream(v, w)
+        v = _golden_values(spec, w)
         if expected == "-":
             want = b""
         elif expected == "literal":
             want = bytes([4, 0]) + v.astype("<u2" if w == 2 else "u1").tobytes()
         else:
-            want = bytes(int(t, 16) for t in expected.split())
-        assert got == want, name
-        rc, back = O.decode_stream(got, w)
+            want = _golden_bytes(expected)
+        rc, back = O.decode_stream(want, w)
         assert rc == 0 and (back == v).all(), name
+        got = O.encode_stream(v, w)
+        if name.startswith("dec_"):
+            assert got != want, name                      # the encoder picks shift 0 for these
+            assert O.stream_header(got)[2] == 0, name
+            rc, back = O.decode_stream(got, w)
+            assert rc == 0 and (back == v).all(), name
+        else:
+            assert got == want, name
+        seen.add(name.split("_")[0])
+    assert {"empty", "const", "sparse", "literal", "paired", "based", "dec"} <= seen
 
 
 # ----------------------------------------------------------------------------
@@ -224,6 +267,87 @@ def test_model_choice_near_best():
             tot_sel += sel
             tot_best += best
     assert tot_sel <= 1.01 * tot_best
+
+
+def _brute_model(hist, box, cost):
+    """Spec S6 by enumeration: among the models whose box holds the largest hi,
+    the lowest total fixed-point cost sum_v h[v] * cost[m][v]; ties to the lowest m."""
+    top = max(v for v in range(16) if hist[v])
+    best_m, best_c = None, None
+    for m in range(32):
+        if box[m] < top:
+            continue
+        total = sum(int(hist[v]) * int(cost[m][v]) for v in range(16) if hist[v])
+        if best_c is None or total < best_c:
+            best_m, best_c = m, total
+    return best_m
+
+
+def _tie_histograms(box, cost):
+    """Histograms over hi in {0, 1, 2} (512 counts) on which two models reach the
+    lowest total exactly: the rule must pick the lower model number."""
+    out = []
+    for h1 in range(0, 513, 3):
+        for h2 in range(1, 513 - h1):
+            h0 = 512 - h1 - h2
+            if h0 < 1:
+                continue
+            tot = {m: h0 * int(cost[m][0]) + h1 * int(cost[m][1]) + h2 * int(cost[m][2])
+                   for m in range(32) if box[m] >= 2}
+            low = min(tot.values())
+            if sum(1 for t in tot.values() if t == low) > 1:
+                out.append((h0, h1, h2))
+    return out
+
+
+def test_model_choice_exact():
+    """Spec S6 model selection against enumeration over all 32 frozen models: random
+    hi histograms (with and without base and raw low bits) and constructed exact ties,
+    which must go to the lowest model number."""
+    _, _, box, cost = frozen_tables()
+    rng = np.random.default_rng(31)
+    cases = []
+    for lam in [0.01, 0.05, 0.2, 0.7, 1.5, 3, 6, 10, 14]:
+        for _ in range(6):
+            v = np.minimum(rng.poisson(lam, 512), 15)
+            v[rng.integers(0, 512)] = 0                 # min 0: no base, shift 0
+            if v.max() > 0:
+                cases.append(("plain", v.astype(np.uint16), 1))
+    for _ in range(20):                                 # base and raw low bits (uint16)
+        base = int(rng.integers(1, 3000))
+        shift = int(rng.integers(1, 9))
+        hi = np.minimum(rng.poisson(rng.uniform(0.2, 9), 512), 15)
+        hi[rng.integers(0, 512)] = 0
+        hi[rng.integers(0, 512)] = max(8, int(hi.max()))   # top hi >= 8 keeps the shift
+        lo = rng.integers(0, 1 << shift, 512)
+        lo[hi.argmin()] = 0                             # one element equals the base
+        cases.append(("shifted", (base + (hi << shift) + lo).astype(np.uint16), 2))
+    ties = _tie_histograms(box, cost)
+    assert len(ties) >= 20
+    for h0, h1, h2 in ties[:: max(1, len(ties) // 24)]:
+        v = np.array([0] * h0 + [1] * h1 + [2] * h2, np.uint16)
+        cases.append(("tie", rng.permutation(v), 1))
+    n_ties = 0
+    for kind, v, w in cases:
+        vv = v.astype(np.int64)
+        base = int(vv.min())
+        shift = max(0, int(vv.max() - base).bit_length() - 4)
+        hist = np.bincount((vv - base) >> shift, minlength=16)
+        want = _brute_model(hist, box, cost)
+        got = O.stream_sizes(v, w)[3]
+        assert got == want, (kind, hist.tolist(), got, want)
+        if kind == "tie":
+            top = max(t for t in range(16) if hist[t])
+            lows = [m for m in range(32) if box[m] >= top and
+                    sum(int(hist[t]) * int(cost[m][t]) for t in range(16)) ==
+                    sum(int(hist[t]) * int(cost[want][t]) for t in range(16))]
+            assert len(lows) > 1 and want == min(lows)
+            n_ties += 1
+        s = O.encode_stream(v, w)
+        hdr = O.stream_header(s)
+        if hdr[0] == 3:
+            assert hdr[1] == want and hdr[2] == shift and hdr[3] == int(base > 0)
+    assert n_ties >= 20
 
 
 @pytest.mark.parametrize("w", [1, 2])

@@ -31,7 +31,8 @@ def sources() -> list[str]:
 def stale() -> bool:
     if not os.path.exists(LIB):
         return True
-    deps = sources() + glob.glob(os.path.join(SRC_DIR, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    deps = (sources() + glob.glob(os.path.join(SRC_DIR, "*.h")) + glob.glob(os.path.join(SRC_DIR, "*.inc")) +
+            glob.glob(os.path.join(INCLUDE, "*.h")))
     return max(os.path.getmtime(p) for p in deps) > os.path.getmtime(LIB)
 
 

@@ -2,20 +2,22 @@
 //
 // Page "Paired-count resident layout", "Operation pipeline" step 2: each
 // stream is coded with "a 1024-state tANS table from 32 Poisson pair models".
-// The models, quantisation and spread are the library's spec S4/S5; tANS is
-// Duda's tabled asymmetric numeral systems (arXiv:1311.2540).  The tables are
-// computed once per process in IEEE double, in the evaluation order the spec
-// writes down, then packed for the device kernels.
-#include <algorithm>
+// The models and their quantisation are the library's spec S4; tANS is
+// Duda's tabled asymmetric numeral systems (arXiv:1311.2540), with the spread
+// of spec S5.  Page "Contract": the coding parameters are fixed by the ABI
+// string.  So the S4 results (frequencies, box sizes, selection costs) are
+// frozen integer data (model_tables.inc, written once by
+// gen_model_tables.cpp) and everything derived here from them is integer
+// arithmetic: no libm call can move a table from one host to another.
 #include <array>
-#include <cmath>
 #include <mutex>
-#include <vector>
 
 #include "qem_internal.h"
 
 namespace qem {
 namespace {
+
+#include "model_tables.inc"
 
 constexpr int kSpreadStep = 643;   // (5/8)L + 3, odd, so the walk covers all 1024 slots
 
@@ -31,67 +33,12 @@ int floor_log2(int y)
 
 void make_model(int m, HostTables &T)
 {
-    const double lambda = 0.005 * std::pow(3200.0, static_cast<double>(m) / 31.0);
-
-    // Poisson(lambda) on 0..14 by the pmf recurrence; the tail is folded into 15.
-    std::array<double, 16> q{};
-    q[0] = std::exp(-lambda);
-    for (int v = 1; v <= 14; ++v)
-        q[v] = (q[v - 1] * lambda) / static_cast<double>(v);
-    double head = 0.0;
-    for (int v = 0; v <= 14; ++v)
-        head += q[v];
-    q[15] = std::max(0.0, 1.0 - head);
-
-    // The model's box 0..A: the first A whose remaining mass is below 2^-20.
-    int A = 15;
-    for (int cand = 0; cand < 15; ++cand) {
-        double rest = 0.0;
-        for (int v = cand + 1; v <= 15; ++v)
-            rest += q[v];
-        if (rest < 1.0 / 1048576.0) {
-            A = cand;
-            break;
-        }
-    }
-    T.amax[m] = static_cast<uint8_t>(A);
-
-    double mass = 0.0;
-    for (int v = 0; v <= A; ++v)
-        mass += q[v];
-    std::array<double, 16> t{};
-    for (int v = 0; v <= A; ++v)
-        t[v] = q[v] / mass;
-
+    // The model's frequencies, box and selection costs are the frozen S4 data.
+    for (int s = 0; s < 256; ++s)
+        T.freq[m][s] = kFreq[m][s];
+    T.amax[m] = kBox[m];
     for (int v = 0; v < 16; ++v)
-        T.cost[m][v] = v <= A ? static_cast<uint32_t>(std::floor(-256.0 * std::log2(t[v]) + 0.5))
-                              : 0xFFFFFFFFu;
-
-    // Frequencies: one reserved slot per box symbol, floor of the scaled rest,
-    // then the leftover units to the largest fractional parts (lower symbol first).
-    const int boxed = (A + 1) * (A + 1);
-    const double scale = static_cast<double>(kStates - boxed);
-    struct Cand {
-        double frac;
-        int sym;
-    };
-    std::vector<Cand> order;
-    int used = 0;
-    for (int s = 0; s < 256; ++s) {
-        const int a = s & 15, b = s >> 4;
-        T.freq[m][s] = 0;
-        if (a > A || b > A)
-            continue;
-        const double scaled = (t[a] * t[b]) * scale;
-        const double whole = std::floor(scaled);
-        T.freq[m][s] = static_cast<uint16_t>(1 + static_cast<int>(whole));
-        used += T.freq[m][s];
-        order.push_back({scaled - whole, s});
-    }
-    std::stable_sort(order.begin(), order.end(),
-                     [](const Cand &x, const Cand &y) { return x.frac > y.frac; });
-    for (int k = 0; k < kStates - used; ++k)
-        T.freq[m][order[k].sym] += 1;
+        T.cost[m][v] = kCost[m][v];
 
     // Spread symbols over the slots with the odd step, ascending symbol order.
     std::array<uint8_t, kStates> slot_sym{};
