@@ -266,6 +266,22 @@ def dense_masked_sum(counts: np.ndarray, mask: np.ndarray, valid: np.ndarray | N
     return out
 
 
+def dense_block_sums(counts_block: np.ndarray, masks, valid: np.ndarray | None = None) -> np.ndarray:
+    """Plain definition for one 512-scan block and several masks at once:
+    V[m][i] = sum over p with masks[m][p] & valid[p] of x[i][p] (uint64 [n_masks][512]).
+
+    Written as one matrix product x[512][P] @ S[P][n_masks] in float64 (a library
+    primitive standing for the sums): every partial sum is an integer below
+    P * 65535 < 2^53, so each float64 addition is exact and the order of the
+    additions cannot change the result."""
+    sel = np.asarray(masks, dtype=bool).reshape(-1, counts_block.shape[1])
+    if valid is not None:
+        sel = sel & valid.astype(bool)[None, :]
+    assert counts_block.shape[1] * 65535 < 2 ** 53
+    out = counts_block.astype(np.float64) @ sel.T.astype(np.float64)
+    return np.rint(out.T).astype(np.uint64)
+
+
 def dense_masked_moments(counts: np.ndarray, mask: np.ndarray, weights: np.ndarray,
                          valid: np.ndarray | None = None, k: int = 1) -> np.ndarray:
     """Plain definition of the fused moment reduction (page "Backend Optimization Matrix",
@@ -290,6 +306,14 @@ def dense_masked_moments(counts: np.ndarray, mask: np.ndarray, weights: np.ndarr
 
 def dense_decode_blocks(counts: np.ndarray, first: int, n: int, valid: np.ndarray | None = None):
     out = counts[first * 512:(first + n) * 512].copy()
+    if valid is not None:
+        out[:, ~valid.astype(bool)] = 0
+    return out
+
+
+def dense_decode_range(counts: np.ndarray, first_scan: int, n_scans: int, valid: np.ndarray | None = None):
+    """Plain definition of a scan-range decode: out[i][p] = valid[p] ? x[first_scan + i][p] : 0."""
+    out = counts[first_scan:first_scan + n_scans].copy()
     if valid is not None:
         out[:, ~valid.astype(bool)] = 0
     return out

@@ -457,6 +457,24 @@ def test_masked_sum_equals_dense(name):
         assert (frames[:, valid == 1] == x[:512][:, valid == 1]).all()
 
 
+def test_dense_block_sums_is_the_masked_sum():
+    """The many-mask form of the plain definition equals the per-mask one, on random
+    masks and counts, with invalid pixels, and at the largest sums it is used for
+    (a full 192x192 detector of 65535)."""
+    rng = np.random.default_rng(12)
+    for P, w in [(97, 8), (1000, 16)]:
+        x = rng.integers(0, 1 << w, size=(512, P)).astype(np.uint8 if w == 8 else np.uint16)
+        masks = (rng.random((7, P)) < rng.random((7, 1))).astype(np.uint8)
+        valid = (rng.random(P) < 0.9).astype(np.uint8)
+        got = O.dense_block_sums(x, masks, valid)
+        for m in range(7):
+            assert (got[m] == O.dense_masked_sum(x, masks[m], valid)[0]).all()
+    x = np.full((512, 192 * 192), 65535, np.uint16)
+    x[::5, ::7] = 1
+    full = np.ones((1, 192 * 192), np.uint8)
+    assert (O.dense_block_sums(x, full)[0] == x.astype(np.uint64).sum(axis=1)).all()
+
+
 def test_uint64_promotion_257():
     """Contract: uint64 when a full-detector sum could exceed 2**32 (257x257 uint16)."""
     c = _contract()

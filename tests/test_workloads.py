@@ -66,3 +66,16 @@ def test_counter_regeneration_is_positional():
     assert (a[100:150] == b).all()
     uni = w.counter.class_desc[w.counter.pixel_class][:, 0] == W.KIND_UNIFORM
     assert int(uni.sum()) == 184
+
+
+def test_c_generator_equals_numpy_generator():
+    """The C host generator (used to regenerate whole full-size acquisitions for the
+    parity tests) gives the NumPy generator's counts bit for bit, on scans from the
+    start, the middle and the end of every counter workload."""
+    assert W._cgen_lib() is not None, "counter_gen.c did not build"
+    for name in ("c3", "c4", "c5"):
+        w = W.workload(name)
+        for s0 in (0, 511, w.n_scans // 2 + 3, w.n_scans - 6):
+            a = W.counter_counts(w.counter, s0, 6)
+            b = W.counter_counts_fast(w.counter, s0, 6)
+            assert a.dtype == b.dtype and (a == b).all(), (name, s0)
