@@ -1,4 +1,4 @@
-"""CPU oracle for the paired-count resident (qem-pair-v1).
+"""CPU oracle for the paired-count resident (qem-pair-v2).
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 bench's ``cpu_baseline`` / ``--impl reference`` leg may import this package.
@@ -90,7 +90,7 @@ def _ptr(a: np.ndarray):
 
 
 class MalformedStream(ValueError):
-    """A stream failed a qem-pair-v1 check (the query returns no result)."""
+    """A stream failed a qem-pair-v2 check (the query returns no result)."""
 
 
 # ----------------------------------------------------------------------------

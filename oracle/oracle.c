@@ -1,5 +1,5 @@
 /*
- * oracle.c -- plain CPU oracle for the paired-count resident (qem-pair-v1).
+ * oracle.c -- plain CPU oracle for the paired-count resident (qem-pair-v2).
  *
  * TEST INFRASTRUCTURE ONLY (see oracle.h).  Nothing here is used by the CUDA
  * library; the library implements the same written specification on its own.
@@ -9,7 +9,7 @@
  * constant / sparse / incompressible forms, grouped offsets) and section
  * "Contract" (2-byte stream header, sparse preferred unless the paired stream
  * saves at least two bytes; malformed streams raise).  Where the pages leave
- * the format open, this file follows the build's own qem-pair-v1 spec, whose
+ * the format open, this file follows the build's own qem-pair-v2 spec, whose
  * numbered sections are cited below as "spec S<n>".
  */
 #include "oracle.h"
@@ -22,6 +22,9 @@
 #define NMODEL 32            /* Poisson pair models (pages: 32)               */
 #define NPAIR 256            /* 512 scans -> 256 consecutive count pairs      */
 #define SPREAD_STEP 643      /* spec S5: odd step 5L/8 + 3                     */
+#define ONE_STATE_MODELS 8   /* spec S3/S5: models 0-7 code a paired stream with one
+                                tANS state; models 8-31 with two interleaved states
+                                (state A for even pairs, B for odd pairs)        */
 
 #define FORM_CONSTANT 1
 #define FORM_SPARSE 2
@@ -273,20 +276,23 @@ static int encode_paired(const uint16_t v[512], int w, uint8_t *out, int force_m
         }
     }
 
-    /* tANS over pairs 255..0, starting from state 1024 */
+    /* tANS over pairs 255..0, every state starting from 1024; with two states,
+       pair j is coded on state j & 1 */
     uint32_t chunk_v[NPAIR];
     int chunk_n[NPAIR];
-    uint32_t X = NSTATE;
+    int two = model >= ONE_STATE_MODELS;
+    uint32_t X[2] = {NSTATE, NSTATE};
     for (j = NPAIR - 1; j >= 0; j--) {
+        int q = two ? (j & 1) : 0;
         int s = (int)(hi[2 * j] + 16u * hi[2 * j + 1]);
         uint32_t f = M.freq[model][s];
         int k = 0;
-        while ((X >> k) >= 2 * f)
+        while ((X[q] >> k) >= 2 * f)
             k++;
-        chunk_v[j] = X & ((1u << k) - 1u);
+        chunk_v[j] = X[q] & ((1u << k) - 1u);
         chunk_n[j] = k;
-        uint32_t y = X >> k;
-        X = NSTATE + M.sorted_slot[model][M.cum[model][s] + (y - f)];
+        uint32_t y = X[q] >> k;
+        X[q] = NSTATE + M.sorted_slot[model][M.cum[model][s] + (y - f)];
     }
 
     *model_out = model;
@@ -304,7 +310,9 @@ static int encode_paired(const uint16_t v[512], int w, uint8_t *out, int force_m
         put_bits(out + off, &pos, lo[e], shift);
     off += 64 * shift;
     pos = 0;
-    put_bits(out + off, &pos, X - NSTATE, 10);
+    put_bits(out + off, &pos, X[0] - NSTATE, 10);
+    if (two)
+        put_bits(out + off, &pos, X[1] - NSTATE, 10);
     for (j = 0; j < NPAIR; j++)
         put_bits(out + off, &pos, chunk_v[j], chunk_n[j]);
     return off + (int)((pos + 7) / 8);
@@ -333,7 +341,7 @@ void orc_encode_stream(const uint16_t v[512], int w, uint8_t *out, int *len)
     }
     int s_lit = 2 + 512 * w;
     int s_sparse = n <= 256 ? 3 + (9 * n + 7) / 8 + n * w : 1 << 30;
-    uint8_t paired[2 + 2 + 64 * 12 + 330];
+    uint8_t paired[2 + 2 + 64 * 12 + 332];
     memset(paired, 0, sizeof(paired));
     int model;
     int s_paired = encode_paired(v, w, paired, -1, &model);
@@ -465,11 +473,18 @@ int orc_decode_stream(const uint8_t *s, int len, int w, uint16_t v[512])
     const uint8_t *ts = s + off;
     long limit = 8L * (len - off);
     long pos = 0;
-    long x0 = get_bits(ts, &pos, 10, limit);
-    uint32_t X = NSTATE + (uint32_t)x0;
+    int two = model >= ONE_STATE_MODELS;
+    uint32_t X[2] = {NSTATE, NSTATE};
+    for (int q = 0; q < 1 + two; q++) {
+        long x0 = get_bits(ts, &pos, 10, limit);
+        if (x0 < 0)
+            return ORC_BAD_LENGTH;
+        X[q] = NSTATE + (uint32_t)x0;
+    }
     uint32_t hi[512];
     for (j = 0; j < NPAIR; j++) {
-        int slot = (int)(X - NSTATE);
+        int q = two ? (j & 1) : 0;
+        int slot = (int)(X[q] - NSTATE);
         int sym = M.dsym[model][slot];
         int nb = M.dnb[model][slot];
         long bits = get_bits(ts, &pos, nb, limit);
@@ -477,9 +492,9 @@ int orc_decode_stream(const uint8_t *s, int len, int w, uint16_t v[512])
             return ORC_BAD_LENGTH;
         hi[2 * j] = (uint32_t)(sym & 15);
         hi[2 * j + 1] = (uint32_t)(sym >> 4);
-        X = NSTATE + M.dnewbase[model][slot] + (uint32_t)bits;
+        X[q] = NSTATE + M.dnewbase[model][slot] + (uint32_t)bits;
     }
-    if (X != NSTATE)
+    if (X[0] != NSTATE || X[1] != NSTATE)
         return ORC_BAD_STATE;
     if ((pos + 7) / 8 != len - off)
         return ORC_BAD_LENGTH;
@@ -606,7 +621,7 @@ int orc_decode_block(const uint32_t *groups, const uint8_t *payload, uint64_t le
 int orc_paired_size(const uint16_t v[512], int w, int model)
 {
     ensure_models();
-    uint8_t buf[2 + 2 + 64 * 12 + 330];
+    uint8_t buf[2 + 2 + 64 * 12 + 332];
     int m;
     memset(buf, 0, sizeof(buf));
     return encode_paired(v, w, buf, model, &m);
@@ -615,7 +630,7 @@ int orc_paired_size(const uint16_t v[512], int w, int model)
 void orc_stream_sizes(const uint16_t v[512], int w, int32_t info[4])
 {
     ensure_models();
-    uint8_t buf[2 + 2 + 64 * 12 + 330];
+    uint8_t buf[2 + 2 + 64 * 12 + 332];
     int e, n = 0, m = -1;
     for (e = 0; e < 512; e++)
         n += v[e] != 0;

@@ -1,5 +1,5 @@
 /*
- * oracle.h -- CPU oracle for the paired-count resident (qem-pair-v1).
+ * oracle.h -- CPU oracle for the paired-count resident (qem-pair-v2).
  *
  * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
  * bench's cpu_baseline / reference leg may load or call this code.  It shares

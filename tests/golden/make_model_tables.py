@@ -3,7 +3,7 @@
 pipeline" step 2: a 1024-state tANS table from 32 Poisson pair models;
 section "Contract": the coding parameters are fixed by the ABI string).
 
-The file freezes the models of the bitstream qem-pair-v1: per model its box
+The file freezes the models of the bitstream qem-pair-v2: per model its box
 (largest codable count), its 16 selection costs and its 256 pair frequencies,
 plus the SHA-256 of their canonical bytes:
 
@@ -40,7 +40,7 @@ def main() -> None:
     freq, box, cost = O.models()
     digest = hashlib.sha256(canonical_bytes(freq, box, cost)).hexdigest()
     lines = [
-        "# Frozen pair models of qem-pair-v1 (spec S4), written by make_model_tables.py from the oracle.",
+        "# Frozen pair models of qem-pair-v2 (spec S4), written by make_model_tables.py from the oracle.",
         "# Page \"Paired-count resident layout\", Operation pipeline step 2 (32 Poisson pair models,",
         "# 1024-state tANS) and Contract (coding parameters fixed by the ABI string).",
         "# sha256 covers freq <u2 [32][256] | box u1 [32] | cost <u4 [32][16], in that order.",

@@ -243,8 +243,9 @@ def test_tans_cost_matches_shannon():
                     continue
                 hdr = O.stream_header(O.encode_stream(v, 1))
                 shift = 0
-                ideal = 10 + sum(math.log2(1024 / f[m][int(v[2 * j] + 16 * v[2 * j + 1])])
-                                 for j in range(256))
+                states = 2 if m >= 8 else 1              # spec S3: models 8-31 use two states
+                ideal = 10 * states + sum(math.log2(1024 / f[m][int(v[2 * j] + 16 * v[2 * j + 1])])
+                                          for j in range(256))
                 bits_hi = 8 * (n - 2 - 64 * shift)
                 # tANS tracks the Shannon length of its quantised model to within
                 # the initial state plus a few percent (slot-position error)
