@@ -77,20 +77,33 @@ def stream_lengths(res, w):
     return lens
 
 
-def decompose(slots, roots, P, add, rem):
+PLAN_HEAVY, PLAN_LIGHT, PLAN_ITEM = 16, 1, 2     # the index plan's planner weights
+
+
+def decompose(slots, roots, P, add, rem, pclass=None):
     """The plan's split of a query over the index layout: (items, residual pixels).
     add/rem: bool [P] pixels entering / leaving the image (a full query has no rem).
     Items are (level, id): a leaf whose every pixel enters (or every pixel leaves), or a
-    root whose leaves all do so in the same direction."""
+    root whose leaves all do so in the same direction.  In a full query with the pixel
+    classes given, a leaf partly in the mask becomes an item plus its unmasked pixels
+    (subtracted) when their decode weight plus PLAN_ITEM is below the masked pixels'
+    (heavy pixels PLAN_HEAVY, light ones PLAN_LIGHT).  The residual pixels are decoded
+    (added or subtracted); the first return holds the items."""
     real = slots < P
     px = np.where(real, slots, 0)
     a = np.where(real, add[px], True).all(axis=1)
     r = np.where(real, rem[px], True).all(axis=1) & rem.any()
     state = np.where(a, 1, np.where(r, 2, 0))
+    if pclass is not None and not rem.any():
+        wgt = np.where(pclass[px] != 0, PLAN_LIGHT, PLAN_HEAVY) * real
+        inside = add[px] & real
+        c_in = (wgt * inside).sum(axis=1)
+        c_out = (wgt * (real & ~inside)).sum(axis=1)
+        state = np.where((state == 0) & (PLAN_ITEM + c_out < c_in), 3, state)
     items, covered = [], np.zeros(slots.shape[0], bool)
     for i in range(len(roots) - 1):
         s = state[roots[i]:roots[i + 1]]
-        if s[0] > 0 and (s == s[0]).all():
+        if s[0] in (1, 2) and (s == s[0]).all():
             items.append((1, i))
             covered[roots[i]:roots[i + 1]] = True
         else:
@@ -101,7 +114,12 @@ def decompose(slots, roots, P, add, rem):
     cov = np.zeros(P, bool)
     cov[slots[covered][slots[covered] < P]] = True
     resid = (add | rem) & ~cov
-    return items, resid
+    # leaves taken as item minus their unmasked pixels
+    comp = np.zeros(P, bool)
+    for l in np.nonzero(state == 3)[0]:
+        q = slots[l][slots[l] < P]
+        comp[q[~add[q]]] = True
+    return items, resid | comp
 
 
 def algorithmic_bytes(lens, w, sched, out_bits, idx=None):
@@ -123,8 +141,8 @@ def algorithmic_bytes(lens, w, sched, out_bits, idx=None):
         items = []
         resid = add | rem
         if idx is not None and not as_delta:           # deltas take the per-pixel plan
-            slots, roots, gbytes = idx
-            items, resid = decompose(slots, roots, w.n_pixels, add, rem)
+            slots, roots, gbytes, pclass = idx
+            items, resid = decompose(slots, roots, w.n_pixels, add, rem, pclass)
         pix = np.nonzero(resid)[0]
         enc = int(lens[rows][:, pix].sum(dtype=np.int64))
         groups = len(np.unique(pix // 32)) * len(rows)
@@ -280,42 +298,88 @@ def build_resident(w, dev, torch, V, stream=None):
     return res, buf, t_enc
 
 
-def cpu_baseline(w, sample_blocks=4):
-    """The oracle as it stands, on the host cores: BF and ADF k=1 queries over a sample of blocks,
-    scaled to the full acquisition."""
+def oracle_sample(w, n_blocks=4):
+    """The oracle's sample of a workload: n_blocks blocks spread evenly over the
+    acquisition (block i * B / n), regenerated on the host and encoded by the oracle.
+    Returns (blocks, Encoded, encode seconds on all cores, encode seconds on one core
+    for the first block)."""
     import oracle as O
 
-    blocks = list(range(0, w.n_blocks, max(1, w.n_blocks // sample_blocks)))[:sample_blocks]
+    blocks = sorted({int(i * w.n_blocks // n_blocks) for i in range(n_blocks)})
     counts = [w.block_counts(b) for b in blocks]
-    enc = O.Encoded(w.n_pixels, w.dtype_bits)
-    for c in counts:
-        g, p = O.encode_block(c, w.dtype_bits)
-        enc.groups.append(g)
-        enc.payloads.append(p)
+    threads = os.cpu_count() or 1
+    enc = O.Encoded(w.n_pixels, w.dtype_bits, [None] * len(blocks), [None] * len(blocks))
+
+    def job(i):
+        enc.groups[i], enc.payloads[i] = O.encode_block(counts[i], w.dtype_bits)
+
+    from concurrent.futures import ThreadPoolExecutor
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(min(threads, len(blocks))) as ex:
+        list(ex.map(job, range(len(blocks))))
+    t_all = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    O.encode_block(counts[0], w.dtype_bits)
+    t_one = time.perf_counter() - t1
+    return blocks, enc, t_all, t_one
+
+
+def oracle_step(w, enc, n_sample, sched, threads):
+    """One step of the schedule by the oracle over the sampled blocks: every query runs
+    over them (a delta from the previous query's image) and its time per block is scaled
+    to the ceil(B/k) blocks the query touches in the full acquisition.  Returns the scaled
+    step time in seconds and the raw bytes the step's queries cover."""
+    import oracle as O
+
+    prev = img = None
+    scaled = 0.0
+    raw = 0
+    w_bytes = w.dtype_bits // 8
+    for label, m, k, delta in sched:
+        t0 = time.perf_counter()
+        if delta and prev is not None:
+            img = O.resident_delta(enc, img, prev, m, None, 1, threads=threads)
+        else:
+            img = O.resident_masked_sum(enc, m, None, 1, threads=threads)
+        scaled += (time.perf_counter() - t0) / n_sample * math.ceil(w.n_blocks / k)
+        raw += int((m != 0).sum()) * 512 * math.ceil(w.n_blocks / k) * w_bytes
+        prev = m
+    return scaled, raw
+
+
+SAMPLE_RULE = ("every query of the step runs over {n} blocks spread evenly over the acquisition ({blocks} of {B}, "
+               "regenerated on the host and encoded by the oracle) and its time per block is scaled to the "
+               "ceil(B/k) blocks it touches; encode time of the same blocks scaled to all B blocks")
+
+
+def cpu_baseline(w, min_seconds=10.0):
+    """The oracle as it stands, on the host cores, with the reference arm's sampling rule:
+    queries/s of the step's schedule, raw-equivalent GB/s of those queries, encode GB/s,
+    each also on one core."""
+    blocks, enc, t_enc, t_enc_one = oracle_sample(w)
+    sched = schedule(w)
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    n = 0
+    steps = scaled = raw = 0
     while True:
-        for name in ("bf", "adf"):
-            O.resident_masked_sum(enc, w.masks[name], None, 1, threads=threads)
-            n += 1
-        if time.perf_counter() - t0 > 10.0:
+        s_, r_ = oracle_step(w, enc, len(blocks), sched, threads)
+        steps += 1
+        scaled += s_
+        raw = r_
+        if time.perf_counter() - t0 > min_seconds:
             break
-    dt = (time.perf_counter() - t0) / n
-    full = dt * w.n_blocks / len(blocks)
-    # the same queries on one core, over one block
-    one = O.Encoded(w.n_pixels, w.dtype_bits)
-    one.groups.append(enc.groups[0])
-    one.payloads.append(enc.payloads[0])
-    t1 = time.perf_counter()
-    for name in ("bf", "adf"):
-        O.resident_masked_sum(one, w.masks[name], None, 1, threads=1)
-    single = (time.perf_counter() - t1) / 2 * w.n_blocks
-    return {"value": 1.0 / full, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu": cpu_model(),
-            "single_core_value": 1.0 / single,
-            "sample": f"bf/adf k=1 queries over {len(blocks)} of {w.n_blocks} blocks (host-regenerated), "
-                      f"{n} queries in {dt * n:.1f} s, scaled to all blocks; single core: one bf and one adf "
-                      f"query over block {blocks[0]}, scaled the same way"}
+    wall = time.perf_counter() - t0
+    step_s = scaled / steps
+    one_s, _ = oracle_step(w, enc, len(blocks), sched, 1)
+    block_raw = 512 * w.n_pixels * (w.dtype_bits // 8)
+    return {"value": len(sched) / step_s, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu": cpu_model(),
+            "raw_equiv_gbs": raw / step_s / 1e9,
+            "encode_gbs": block_raw * len(blocks) / t_enc / 1e9,
+            "single_core": {"value": len(sched) / one_s, "raw_equiv_gbs": raw / one_s / 1e9,
+                            "encode_gbs": block_raw / t_enc_one / 1e9},
+            "sample": SAMPLE_RULE.format(n=len(blocks), blocks=blocks, B=w.n_blocks)
+                      + f"; {steps} steps in {wall:.1f} s of CPU time on {threads} threads"}
 
 
 def cpu_model():
@@ -361,48 +425,37 @@ def workload_config(w, nq, world):
 
 
 def run_reference(args, rank, world):
-    """The oracle timed on the host cores on a bounded sample (2 blocks) of the same workload and schedule:
-    every query of the step runs over the sampled blocks, and its time per block is scaled by the number
-    of blocks the query touches in the full acquisition (ceil(B/k))."""
-    import oracle as O
-
+    """The oracle timed on the host cores on a bounded sample of the same workload and
+    schedule (the sampling rule of SAMPLE_RULE, the same as the cpu_baseline leg)."""
     if rank != 0:
         return
     w = W.workload(args.config)
-    blocks = [0, w.n_blocks // 2]
-    enc = O.Encoded(w.n_pixels, w.dtype_bits)
-    for b in blocks:
-        g, p = O.encode_block(w.block_counts(b), w.dtype_bits)
-        enc.groups.append(g)
-        enc.payloads.append(p)
+    blocks, enc, t_enc, _ = oracle_sample(w)
     sched = schedule(w)
     threads = os.cpu_count() or 1
-
-    def step():
-        prev = img = None
-        scaled = 0.0
-        for label, m, k, delta in sched:
-            t0 = time.perf_counter()
-            if delta and prev is not None:
-                img = O.resident_delta(enc, img, prev, m, None, 1, threads=threads)
-            else:
-                img = O.resident_masked_sum(enc, m, None, 1, threads=threads)
-            scaled += (time.perf_counter() - t0) / len(blocks) * math.ceil(w.n_blocks / k)
-            prev = m
-        return scaled
-
     for _ in range(args.warmup):
-        step()
-    step_full = sum(step() for _ in range(args.steps)) / args.steps
+        oracle_step(w, enc, len(blocks), sched, threads)
+    t0 = time.perf_counter()
+    tot = 0.0
+    raw = 0
+    for _ in range(args.steps):
+        s_, raw = oracle_step(w, enc, len(blocks), sched, threads)
+        tot += s_
+    wall = time.perf_counter() - t0
+    step_full = tot / args.steps
     value = len(sched) / step_full
+    sample = (SAMPLE_RULE.format(n=len(blocks), blocks=blocks, B=w.n_blocks)
+              + f"; {args.steps} timed steps took {wall:.1f} s of CPU time; ms_per_step is the scaled "
+                f"full-acquisition step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_full * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u8" if w.dtype_bits == 8 else "u16",
             "data": "synthetic",
             "config": workload_config(w, len(sched), world),
+            "raw_equiv_gbs": raw / step_full / 1e9,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu": cpu_model(),
-                             "sample": f"each of the {len(sched)} queries of a step timed over blocks {blocks} of "
-                                       f"{w.n_blocks} and scaled to the ceil(B/k) blocks it touches"},
+                             "encode_gbs": 512 * w.n_pixels * (w.dtype_bits // 8) * len(blocks) / t_enc / 1e9,
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -439,6 +492,10 @@ def run_profile_case(dev, torch, V):
     for k in (4, 16):
         for m in (bf, adf):
             res.masked_sum(m, block_stride=k, out=out[: -(-w.n_blocks // k)])
+    # a two-block decode and one frame (k_decode_blocks, k_decode_range)
+    frames = torch.empty((2 * 512, w.n_pixels), dtype=torch.uint8, device=dev)
+    res.decode_blocks(0, 2, out=frames)
+    res.decode_range(777, 1)
     p = res.profile_read()
     print(json.dumps({"encode_s": t_enc, "kernels": p}), flush=True)
     res.free()
@@ -721,7 +778,7 @@ def main():
         slots, roots = res.index_layout()
         codes = res.index_desc() >> 30
         gbytes = np.where(codes > 0, 512 << np.maximum(codes.astype(np.int64) - 1, 0), 0)
-        idx = (slots, roots, gbytes)
+        idx = (slots, roots, gbytes, res.pixel_classes())
     ab = algorithmic_bytes(lens, w, sched, out_bits, idx)
     # per query: the median of 20 warm passes over the schedule, each query timed
     # alone (events around the call, synchronised after it)
@@ -746,6 +803,109 @@ def main():
         d["enc_gbs"] = d["enc_bytes"] / (d["ms"] / 1e3) / 1e9
 
     hbm, peak_kind = peaks()
+
+    # single diffraction frames: one-scan range decodes at 20 scans spread over the
+    # acquisition, each timed alone; the first is checked against a block decode
+    odt_counts = torch.uint8 if w.dtype_bits == 8 else torch.uint16
+    fr = torch.empty((1, w.n_pixels), dtype=odt_counts, device=dev)
+    f_scans = [int(x) for x in np.linspace(0, w.n_scans - 1, 20)]
+    res.decode_range(f_scans[0], 1, out=fr)
+    f_exact = bool(torch.equal(fr[0], res.decode_blocks(f_scans[0] // 512, 1)[f_scans[0] % 512]))
+    f_ms = []
+    for sc in f_scans:
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record()
+        res.decode_range(sc, 1, out=fr, wait=False)
+        q1.record()
+        torch.cuda.synchronize()
+        f_ms.append(q0.elapsed_time(q1))
+    res.finish()
+    frame = {"ms": statistics.median(f_ms), "ms_max": max(f_ms), "runs": len(f_ms), "exact": f_exact,
+             "gcounts_per_s": w.n_pixels / (statistics.median(f_ms) / 1e3) / 1e9}
+
+    # dense dark field (every pixel outside the bright-field disk) three ways: the
+    # cached total minus the complement (qem_masked_sum_complement), the interaction
+    # index, and (below, without the index) the plain decode of every masked pixel
+    df_m = torch.from_numpy((1 - w.masks["bf"]).astype(np.uint8)).to(dev)
+    o_df = torch.empty((w.n_blocks, 512), dtype=V.out_dtype(out_bits), device=dev)
+    torch.cuda.synchronize()
+    tb0 = time.perf_counter()
+    res.masked_sum_complement(df_m, out=o_df)
+    t_total_build = time.perf_counter() - tb0
+
+    def med_ms(fn, n=20):
+        xs = []
+        for _ in range(n):
+            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            q0.record()
+            fn()
+            q1.record()
+            torch.cuda.synchronize()
+            xs.append(q0.elapsed_time(q1))
+        res.finish()
+        return statistics.median(xs)
+
+    df_comp = med_ms(lambda: res.masked_sum_complement(df_m, out=o_df, wait=False))
+    img_comp = o_df.clone()
+    df_idx = med_ms(lambda: res.masked_sum(df_m, out=o_df, wait=False))
+    dense_df = {"pixels": int(df_m.sum().item()), "complement_ms": df_comp,
+                "index_ms": df_idx if index is not None else None, "total_build_s": t_total_build,
+                "exact_vs_index": bool(torch.equal(img_comp, o_df))}
+
+    # decode only: the same schedule with the interaction index dropped, so every
+    # masked pixel of every query is decoded (timed without and with per-kernel events,
+    # as `value` and the roofline are), and bf/adf k=1 alone (median of 20)
+    decode_only = None
+    if index is not None:
+        res.drop_index()
+        step()
+        res.finish()
+        torch.cuda.synchronize()
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0.record()
+        for _ in range(args.steps):
+            step()
+        n1.record()
+        torch.cuda.synchronize()
+        res.finish()
+        t_ni = n0.elapsed_time(n1) / 1e3
+        res.profile(True)
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        res.finish()
+        prof_ni = res.profile_read()
+        res.profile(False)
+        ab_ni = algorithmic_bytes(lens, w, sched, out_bits, None)
+        bytes_ni = sum(a["bytes"] for a in ab_ni)
+        n_dni, ms_dni = prof_ni["decode_reduce"]
+        q_ni = {}
+        for (label, m, k, delta), md, a in zip(sched, masks, ab_ni):
+            if label not in ("bf_k1", "adf_k1"):
+                continue
+            qs = []
+            for _ in range(20):
+                q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                q0.record()
+                res.masked_sum(md, block_stride=k, out=outs[k], wait=False)
+                q1.record()
+                torch.cuda.synchronize()
+                qs.append(q0.elapsed_time(q1))
+            res.finish()
+            ms = statistics.median(qs)
+            q_ni[label] = {"ms": round(ms, 4), "runs": len(qs), "enc_gbs": round(a["enc"] / (ms / 1e3) / 1e9, 1),
+                           "hbm_frac_enc": round(a["enc"] / (ms / 1e3) / 1e9 / hbm, 4),
+                           "raw_equiv_gbs": round(a["raw"] / (ms / 1e3) / 1e9, 1)}
+        dense_df["plain_ms"] = med_ms(lambda: res.masked_sum(df_m, out=o_df, wait=False))
+        ach_ni = bytes_ni * args.steps / (ms_dni / 1e3) / 1e9 if ms_dni > 0 else None
+        decode_only = {"value": nq_ * args.steps / t_ni, "unit": UNIT, "ms_per_step": t_ni / args.steps * 1e3,
+                       "queries": q_ni,
+                       "roofline": {"achieved": ach_ni, "peak": hbm, "unit": "GB/s",
+                                    "frac": ach_ni / hbm if ach_ni else None, "kernel": "k_decode_reduce",
+                                    "avg_launch_ms": ms_dni / max(1, n_dni),
+                                    "algorithmic_bytes_per_launch": bytes_ni * args.steps / max(1, n_dni)},
+                       "note": "interaction index dropped: every masked pixel of every query decoded"}
+
     # DRAM traffic per decode launch from a committed ncu capture, if it was taken on
     # this exact kernel source (else null)
     traffic = None
@@ -770,7 +930,13 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u8" if w.dtype_bits == 8 else "u16", "data": "synthetic",
         "config": {**workload_config(w, nq, world),
-                   "l2": f"inputs larger than L2: {bytes_step / 1e9:.2f} GB of encoded streams read per step",
+                   "l2": (f"no flush between steps; each step reads {bytes_step / 1e9:.2f} GB of encoded streams, "
+                          f"offsets, index sums and images ({'above' if bytes_step > 126e6 else 'below'} the 126 MB L2), but single launches read "
+                          f"{min(a['bytes'] for a in ab) / 1e6:.1f}-{max(a['bytes'] for a in ab) / 1e6:.1f} MB "
+                          f"(below it) and consecutive queries share streams (bf at stride 4 and 16 reads a "
+                          f"subset of bf at stride 1; a drag delta's leaving pixels were read by the previous "
+                          f"query), so per-query figures are partly served from L2"),
+                   "launch_bytes_mb": {lbl: round(a["bytes"] / 1e6, 2) for (lbl, _, _, _), a in zip(sched, ab)},
                    "resident_bytes": info["payload_bytes"] + info["group_bytes"], "raw_bytes": w.raw_bytes},
         "raw_equiv_gbs": world * raw_step * args.steps / t / 1e9,
         "e2e": {"value": world * nq * args.steps / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
@@ -800,6 +966,9 @@ def main():
         "moments": mom,
         "decode_blocks": {"blocks": nd, "s": dec_s, "gcounts_per_s": nd * 512 * w.n_pixels / dec_s / 1e9,
                           "exact": ok_frames},
+        "frame": frame,
+        "dense_df": dense_df,
+        "decode_only": decode_only,
         "resident": {"payload_bytes": info["payload_bytes"], "forms": info["form_count"],
                      "bits_per_count": 8 * info["payload_bytes"] / (w.n_scans * w.n_pixels)},
         "clocks": clocks,

@@ -3,7 +3,7 @@
  *
  * A 4D-STEM count acquisition (scan_row, scan_col, det_row, det_col), uint8 or
  * uint16, is held on the GPU entropy-coded as per-pixel 512-scan pair-tANS
- * streams (bitstream spec "qem-pair-v1") and queried without a dense copy.
+ * streams (bitstream spec "qem-pair-v2") and queried without a dense copy.
  * Source: page "Paired-count resident layout" (quantem.gpu developer docs),
  * sections "Operation pipeline" (steps 1-6), "Contract" and "Verification".
  *
@@ -36,7 +36,7 @@ extern "C" {
 typedef enum {
     QEM_OK = 0,
     QEM_ERR_ARG = 1,        /* invalid argument (sizes, dtype, stride, out_bits)    */
-    QEM_ERR_MALFORMED = 2,  /* a decoded stream failed a qem-pair-v1 check: the
+    QEM_ERR_MALFORMED = 2,  /* a decoded stream failed a qem-pair-v2 check: the
                                query's output is not a result (page "Contract":
                                malformed stream -> error, the result is not returned) */
     QEM_ERR_CUDA = 3,       /* a CUDA runtime call failed                            */
@@ -87,7 +87,7 @@ typedef struct {
 #define QEM_K_ENC_COMPACT 6
 #define QEM_K_GENERATE 7
 
-/* ABI string of the bitstream this library writes and reads ("qem-pair-v1").
+/* ABI string of the bitstream this library writes and reads ("qem-pair-v2").
  * Page "Contract": the coding parameters are fixed by the ABI string. */
 const char *qem_abi(void);
 
@@ -149,11 +149,45 @@ int qem_masked_sum_delta(qem_resident *res, const uint8_t *d_new_mask, int32_t b
                          int32_t out_bits, void *d_out, int32_t *out_bits_used, int32_t wait,
                          void *stream);
 
+/* Masked sum by complement (page "Backend Optimization Matrix", CUDA
+ * checkpoint rows: dense dark field as a cached total minus the complement):
+ * d_out = T - (sum over the valid pixels outside the mask), where T is the
+ * resident's cached full-detector image (every valid pixel's stream decoded
+ * once, on the first call, which synchronises `stream` and allocates
+ * B x 512 x 8 bytes, kept until qem_free).  The result equals
+ * qem_masked_sum(d_mask); it decodes the complement's streams instead of the
+ * mask's, so it is the cheaper query for a mask covering most of the
+ * detector.  It does not use the interaction index.  The mask and image become
+ * this stride's delta baseline.  Same d_mask, block_stride, out_bits, d_out
+ * and wait rules as qem_masked_sum; QEM_ERR_MALFORMED (no cache kept) if a
+ * stream failed a check while the total was built. */
+int qem_masked_sum_complement(qem_resident *res, const uint8_t *d_mask, int32_t block_stride,
+                              int32_t out_bits, void *d_out, int32_t *out_bits_used, int32_t wait,
+                              void *stream);
+
 /* Block decode (page "Operation pipeline" step 6, decode_blocks(first,
  * scans), read as first block and block count): d_out [n_blocks*512][pixels]
  * in the native dtype (aligned to it), invalid pixels 0.  Same wait rule as the queries. */
 int qem_decode_blocks(qem_resident *res, int64_t first_block, int64_t n_blocks, void *d_out,
                       int32_t wait, void *stream);
+
+/* Scan-range decode (page "Paired-count resident layout", "Source map":
+ * the decode_range and frame kernels; "Contract": queued queries,
+ * session.frame(..., wait=False); "Verification": every frame compared with
+ * direct sums): d_out [n_scans][pixels] in the native dtype (aligned to it)
+ * receives the counts of scans first_scan .. first_scan + n_scans - 1 (scan
+ * index s = scan_row * scan_cols + scan_col), invalid pixels 0; a single
+ * diffraction frame is n_scans = 1.  The range may cross block boundaries
+ * and must lie inside the blocks encoded so far (QEM_ERR_ARG otherwise).
+ * Each stream is decoded only up to the last pair the range needs, so its
+ * end-of-stream checks (final tANS state, exact section length) are left to
+ * block decodes and queries; everything read is checked (header, fields,
+ * form lengths, sparse order, value range, no read past the stream's
+ * extent) and a failed check gives QEM_ERR_MALFORMED.  Same wait rule as
+ * qem_decode_blocks (wait == 0: errors surface at qem_finish).  Profiled
+ * under QEM_K_DECODE_BLOCKS. */
+int qem_decode_range(qem_resident *res, int64_t first_scan, int64_t n_scans, void *d_out, int32_t wait,
+                     void *stream);
 
 /* Interaction index (page "Operation pipeline" step 3: exact per-scan sums of
  * radial-angular pixel groups, 64-pixel leaves and 16-leaf roots; step 4: a
@@ -295,14 +329,21 @@ void qem_free(qem_resident *res);
  * until the process exits.  Consequences:
  *  - the detector may have at most QEM_NOALLOC_MAX_PIXELS pixels, otherwise
  *    QEM_ERR_ARG is returned and nothing runs;
- *  - all calls share that array: calls whose work overlaps on the GPU (other
- *    streams, other threads) race and give wrong results; serialise them;
- *  - the first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture;
- *  - the call waits for its own work on `stream` and returns
- *    QEM_ERR_MALFORMED if a decoded stream failed a check;
- *  - it neither reads nor updates the per-stride delta baselines.
+ *  - all calls share that array, which keeps the last call's contents (each
+ *    call clears the status and counts it needs before using them): calls
+ *    whose work overlaps on the GPU (other streams, other threads) race and
+ *    give wrong results; serialise them;
+ *  - what could allocate is done once per device when a resident is created
+ *    on it (qem_create, qem_encode, qem_import, qem_load): looking up the
+ *    array's device address (cudaGetSymbolAddress, which also loads the
+ *    library code that holds it), loading the kernels this call launches and
+ *    taking one pinned host word for its status; so even the first call on a
+ *    device allocates nothing (QEM_ERR_CUDA if that set-up had failed);
+ *  - the call waits (bounded, ~60 s, QEM_ERR_TIMEOUT) for its own work on
+ *    `stream` and returns QEM_ERR_MALFORMED if a decoded stream failed a
+ *    check;
+ *  - it neither reads nor updates the per-stride delta baselines, and does not
+ *    use the interaction index (results are the same with or without one).
  * The resident must live on the current device and be complete. */
 int qem_masked_sum_noalloc(qem_resident *res, const uint8_t *d_mask, int32_t block_stride,
                            int32_t out_bits, void *d_out, void *stream);
@@ -326,6 +367,13 @@ int qem_import(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_t d
                int32_t dtype_bits, const uint32_t *h_groups, const uint8_t *h_payload,
                const uint64_t *h_block_off, const uint8_t *h_valid, void *stream,
                qem_resident **out);
+
+/* Each pixel's decode class, as the query plans use it to order their work and
+ * to weigh an index item against residual pixels: h_class (host, n_pixels
+ * bytes) receives 1 for pixels whose block-0 stream is light (empty, sparse,
+ * or paired with a low-dose model and no base or raw bits, decoded by runs)
+ * and 0 for the others (decoded pair by pair).  Synchronises the device. */
+int qem_pixel_classes(const qem_resident *res, uint8_t *h_class);
 
 /* The library's own model tables (spec S4), computed on the host:
  * freq [32][256] uint16, amax [32] uint8, cost [32][16] uint32. */

@@ -18,7 +18,7 @@
 
 int main(void)
 {
-    CHECK(strcmp(qem_abi(), "qem-pair-v1") == 0);
+    CHECK(strcmp(qem_abi(), "qem-pair-v2") == 0);
     CHECK(qem_status_string(QEM_ERR_MALFORMED) != NULL);
 
     /* polar layout of a 17 x 17 detector about its centre: every pixel once */

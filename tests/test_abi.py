@@ -47,7 +47,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_abi_string_and_status_names():
     V = _lib()
-    assert V.abi() == "qem-pair-v1"
+    assert V.abi() == "qem-pair-v2"
     assert V.status_string(V.QEM_ERR_MALFORMED) == "malformed stream"
     assert V.status_string(99) == "unknown status"
 

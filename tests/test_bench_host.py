@@ -27,7 +27,12 @@ def _layout(w):
 
 
 @pytest.mark.parametrize("case", ["bf", "adf", "delta"])
-def test_decompose_partitions_the_query(case):
+@pytest.mark.parametrize("classes", [False, True])
+def test_decompose_partitions_the_query(case, classes):
+    """Items plus signed residual pixels add up to exactly the query, items are
+    disjoint, no whole leaf is left residual, and with pixel classes (the c4 light /
+    heavy split: heavy inside the bright-field disk) a leaf becomes item-minus-rest
+    only when that is cheaper by the planner weights."""
     w = W.workload("c4")
     slots, roots = _layout(w)
     P = w.n_pixels
@@ -36,24 +41,32 @@ def test_decompose_partitions_the_query(case):
         add, rem = new & ~old, old & ~new
     else:
         add, rem = w.masks[case].astype(bool), np.zeros(P, bool)
-    items, resid = bench.decompose(slots, roots, P, add, rem)
+    pclass = (~W.disk(192, 192, 96, 96, 30).astype(bool)).astype(np.uint8) if classes else None
+    items, resid = bench.decompose(slots, roots, P, add, rem, pclass)
     covered = np.zeros(P, np.int64)
+    sign = np.zeros(P, np.int64)
     for lvl, g in items:
         leaves = range(roots[g], roots[g + 1]) if lvl == 1 else [g]
         px = np.concatenate([slots[l][slots[l] < P] for l in leaves])
-        # an item's pixels all enter, or all leave
-        assert add[px].all() or rem[px].all(), (lvl, g)
         covered[px] += 1
+        sign[px] += -1 if (rem.any() and rem[px].all()) else 1
     assert covered.max(initial=0) <= 1                       # items are disjoint
-    assert not (resid & (covered > 0)).any()                  # residual pixels are not in items
-    assert np.array_equal(resid | (covered > 0), add | rem)   # together they are the query
-    # no whole leaf is left in the residual list
+    # residual pixels inside an item leaf are subtracted (not in the query), others added
+    contrib = sign + np.where(resid & (covered > 0), -1, 0) + np.where(resid & (covered == 0), np.where(rem, -1, 1), 0)
+    want = add.astype(np.int64) - rem.astype(np.int64)
+    assert np.array_equal(contrib, want)
     for l in range(slots.shape[0]):
         px = slots[l][slots[l] < P]
         assert not (add[px].all() and resid[px].all())
         assert not (rem.any() and rem[px].all() and resid[px].all())
+        if classes and case != "delta" and covered[px].any() and not add[px].all():
+            wgt = np.where(pclass[px] != 0, bench.PLAN_LIGHT, bench.PLAN_HEAVY)
+            assert bench.PLAN_ITEM + wgt[~add[px]].sum() < wgt[add[px]].sum()
     if case == "adf":
         assert len(items) > 0 and resid.sum() < add.sum() // 3
+    if case == "bf" and classes:
+        # edge leaves of the disk are taken whole: few heavy pixels stay residual
+        assert (resid & (pclass == 0)).sum() < (add & (pclass == 0)).sum() // 10
 
 
 def test_algorithmic_bytes_hand_count():

@@ -206,3 +206,33 @@ def test_c4_index_full_size():
     for b, xb in counts.items():
         assert (img[b] == O.dense_masked_sum(xb, w.drag[8])[0]).all()
     res.free()
+
+
+@pytest.mark.parametrize("name", ["c2", "c1"])
+def test_planner_follows_its_weights(data, name):
+    """The index plan's split follows the planner weights (a pair-by-pair stream 16,
+    a light one 1, an item 2): the streams each query decodes are those the host
+    rule gives (bench.decompose with the library's pixel classes), a leaf mostly in
+    the mask is taken whole minus its other pixels, and the images stay exact."""
+    import bench
+
+    w, x, enc = data(name)
+    res = gpu_encode(w, x)
+    res.build_index(centre(w))
+    slots, roots = res.index_layout()
+    pclass = res.pixel_classes()
+    P = w.n_pixels
+    full = np.ones(P, np.uint8)
+    rng = np.random.default_rng(3)
+    masks = [w.masks["bf"], w.masks["adf"], full, (rng.random(P) < 0.8).astype(np.uint8)]
+    took_complement = False
+    for m in masks:
+        res.counters()
+        got = image(res, m, 1)
+        rows, streams = res.counters()
+        items, resid = bench.decompose(slots, roots, P, m.astype(bool), np.zeros(P, bool), pclass)
+        assert (got == O.dense_masked_sum(x, m)).all()
+        assert streams == int(resid.sum()) * w.n_blocks
+        took_complement |= bool((resid & ~m.astype(bool)).any())
+    assert took_complement
+    res.free()

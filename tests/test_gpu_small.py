@@ -270,3 +270,39 @@ def test_library_tables_equal_oracle():
     f, a, c = V.model_tables()
     f2, a2, c2 = O.models()
     assert (f == f2).all() and (a == a2).all() and (c == c2).all()
+
+
+def test_uint8_warps_with_base_and_raw_bits():
+    """uint8 pixels of the two-state models with a base (every count at least 4) or raw
+    low bits (one count of 16 or more) sit in the same 32-pixel groups as plain ones and
+    run-decoded ones; full queries, strides and delta chains (whose decode adds the base
+    and the raw bits after the table steps) match the plain sums, and the bitstreams the
+    oracle's byte for byte."""
+    rng = np.random.default_rng(77)
+    det, scans = 17, 1024
+    P = det * det
+    lam = rng.uniform(0.5, 4.0, size=P)
+    kind = rng.integers(0, 4, size=P)                     # 0 plain, 1 base, 2 raw bits, 3 low dose
+    lam[kind == 3] = 0.01
+    x = rng.poisson(np.broadcast_to(lam, (scans, P))).astype(np.int64)
+    x[:, kind == 1] += 4
+    rows = rng.integers(0, scans, size=(kind == 2).sum())
+    x[rows, np.nonzero(kind == 2)[0]] = rng.integers(16, 120, size=rows.size)
+    x = np.minimum(x, 255).astype(np.uint8)
+    w = W.Workload("mix8", scans // 32, 32, det, det, 8, 0, "host")
+    hdrs = [O.stream_header(O.encode_stream(x[:512, p], 1)) for p in range(P)]
+    paired = [h for h in hdrs if h is not None and h[0] == 3]
+    assert any(h[3] for h in paired) and any(h[2] for h in paired) and any(h[1] >= 8 and not h[2] and not h[3] for h in paired)
+    res = gpu_encode(w, x)
+    g, pay = res.export_block(1)
+    og, op = O.encode_block(x[512:], 8)
+    assert (g == og).all() and (pay == op).all()
+    drag = [W.disk(det, det, 8, 3 + t, 4) for t in range(11)]
+    for k in (1, 2):
+        for m in (np.ones(P, np.uint8), W.disk(det, det, 8, 8, 5)):
+            assert (image(res, m, k) == O.dense_masked_sum(x, m, None, k)).all()
+        img = image(res, drag[0], k)
+        for t in range(1, len(drag)):
+            img = image(res, drag[t], k, delta=True)
+            assert (img == O.dense_masked_sum(x, drag[t], None, k)).all(), (k, t)
+    res.free()

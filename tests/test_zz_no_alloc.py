@@ -1,12 +1,16 @@
-"""The allocation-free masked sum (qem_masked_sum_noalloc) against qem_masked_sum.
+"""The allocation-free masked sum (qem_masked_sum_noalloc).
 
-Some callers must not allocate device memory while they query (a thread that
-must never block on the CUDA allocator, or code under an allocation budget
-fixed at set-up).  qem_masked_sum_noalloc serves them with a fixed working
-array in the library's device globals.  This test calls it through the C ABI
-and checks that two calls in a row give exactly the images the allocating
-entry point gives.  It lives in its own file that pytest collects last, and
-passes alone in a fresh process as well as after the other tests.
+Some callers must not allocate device memory while they query: a render or
+acquisition thread that must never block on the CUDA allocator (cudaMalloc
+can synchronise the device), or code under a memory budget fixed at set-up.
+qem_masked_sum_noalloc serves them with a fixed working array in the
+library's device globals.  These tests call it through the C ABI and check,
+on two calls in a row, that its images equal both the allocating entry
+point's and the plain masked sums of the counts; that a malformed stream is
+reported; that an indexed resident gives the same images; and that the
+device's free memory does not change across its first calls.  The file is
+collected last and passes alone in a fresh process as well as after the
+other tests.
 """
 import ctypes
 
@@ -14,9 +18,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import virtual_imaging_b200 as V
 import workloads as W
-from qem_testlib import device, gpu_encode, to_dev
+from qem_testlib import device, gpu_encode, oracle_resident, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -28,8 +33,8 @@ def _noalloc(res, mask, k, out_bits, out):
                                           ctypes.c_void_p(out.data_ptr()), stream)
 
 
-@pytest.mark.parametrize("name", ["c1", "c2"])
-def test_noalloc_equals_masked_sum(name):
+@pytest.mark.parametrize("name", ["c1", "c2", "u19"])
+def test_noalloc_equals_masked_sum_and_oracle(name):
     device()
     w = W.workload(name)
     x = w.host_counts()
@@ -40,15 +45,88 @@ def test_noalloc_equals_masked_sum(name):
         rows = -(-w.n_blocks // k)
         for m in masks:
             md = to_dev(m.astype(np.uint8))
-            want = V.as_unsigned(res.masked_sum(md, block_stride=k))
+            want = O.dense_masked_sum(x, m, None, k)
+            lib_img = V.as_unsigned(res.masked_sum(md, block_stride=k)).astype(np.uint64)
+            assert (lib_img == want).all()
             for out_bits in (0, 64):
                 width = bits if out_bits == 0 else 64
                 for call in range(2):                       # two calls in a row share the array
                     out = torch.full((rows, 512), -1, dtype=V.out_dtype(width), device=md.device)
                     assert _noalloc(res, md, k, out_bits, out) == V.QEM_OK
-                    got = V.as_unsigned(out)
-                    assert (got.astype(np.uint64) == want.astype(np.uint64)).all(), (name, k, out_bits, call)
+                    got = V.as_unsigned(out).astype(np.uint64)
+                    assert (got == want).all(), (name, k, out_bits, call)
     res.free()
+
+
+def test_noalloc_allocates_nothing():
+    """The device's free memory is the same before the first call on a new resident
+    and after two calls (outputs allocated beforehand)."""
+    dev = device()
+    w = W.workload("c2")
+    x = w.host_counts()
+    res = gpu_encode(w, x)
+    md = to_dev(w.masks["bf"])
+    outs = [torch.zeros((w.n_blocks, 512), dtype=torch.int32, device=dev) for _ in range(2)]
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for out in outs:
+        assert _noalloc(res, md, 1, 0, out) == V.QEM_OK
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free1 == free0, (free0, free1)
+    want = O.dense_masked_sum(x, w.masks["bf"])
+    for out in outs:
+        assert (V.as_unsigned(out).astype(np.uint64) == want).all()
+    res.free()
+
+
+def test_noalloc_indexed_resident():
+    """With an interaction index built, the call still decodes every masked pixel and
+    gives the plain masked sums."""
+    device()
+    w = W.workload("c2")
+    x = w.host_counts()
+    res = gpu_encode(w, x)
+    res.build_index((48, 48))
+    for m in list(w.masks.values()) + [w.drag[3]]:
+        md = to_dev(m)
+        for call in range(2):
+            out = torch.zeros((w.n_blocks, 512), dtype=torch.int32, device=md.device)
+            assert _noalloc(res, md, 1, 0, out) == V.QEM_OK
+            assert (V.as_unsigned(out).astype(np.uint64) == O.dense_masked_sum(x, m)).all()
+    res.free()
+
+
+def test_noalloc_malformed_stream():
+    """A stream with a reserved header bit set inside the mask gives
+    QEM_ERR_MALFORMED; the next call on an intact resident is exact again (the
+    status lives in the shared array and every call clears it)."""
+    device()
+    w = W.workload("c1")
+    x = w.host_counts()
+    enc = O.encode(x, 8)
+    p = int(np.nonzero(w.masks["bf"])[0][5])
+    g = enc.groups[0]
+    gi, j = divmod(p, 32)
+    ends = [0] + [(int(g[gi, 1 + t // 2]) >> (16 * (t & 1))) & 0xFFFF for t in range(32)]
+    start, end = int(g[gi, 0]) + ends[j], int(g[gi, 0]) + ends[j + 1]
+    assert end - start >= 2
+    bad = enc.payloads[0].copy()
+    bad[start + 1] |= 0x80                                  # reserved header bit 15
+    res_bad = oracle_resident(w, enc, payloads=[bad])
+    res_ok = oracle_resident(w, enc)
+    md = to_dev(w.masks["bf"])
+    out = torch.zeros((1, 512), dtype=torch.int32, device=md.device)
+    assert _noalloc(res_bad, md, 1, 0, out) == V.QEM_ERR_MALFORMED
+    assert _noalloc(res_ok, md, 1, 0, out) == V.QEM_OK
+    assert (V.as_unsigned(out).astype(np.uint64) == O.dense_masked_sum(x, w.masks["bf"])).all()
+    # a mask that leaves the damaged pixel out is exact on the damaged resident
+    m2 = w.masks["bf"].copy()
+    m2[p] = 0
+    assert _noalloc(res_bad, to_dev(m2), 1, 0, out) == V.QEM_OK
+    assert (V.as_unsigned(out).astype(np.uint64) == O.dense_masked_sum(x, m2)).all()
+    res_bad.free()
+    res_ok.free()
 
 
 def test_noalloc_rejects_oversize_and_bad_args():

@@ -1,4 +1,4 @@
-"""B200-native paired-count resident for 4D-STEM counts (bitstream ``qem-pair-v1``).
+"""B200-native paired-count resident for 4D-STEM counts (bitstream ``qem-pair-v2``).
 
 Thin ctypes binding over ``libqem.so`` (declared in ``include/qem.h``): it only
 marshals arguments -- torch tensors become device pointers, the current CUDA
@@ -32,7 +32,8 @@ EXPORTS = ("qem_abi", "qem_status_string", "qem_create", "qem_encode", "qem_enco
            "qem_profile", "qem_profile_read", "qem_free", "qem_block_bytes", "qem_export_block", "qem_import",
            "qem_model_tables", "qem_generate_counts", "qem_masked_sum_noalloc", "qem_build_index",
            "qem_drop_index", "qem_index_layout", "qem_index_desc", "qem_export_valid", "qem_save", "qem_load",
-           "qem_decode_blocks_amplitude", "qem_masked_moments", "qem_polar_layout")
+           "qem_decode_blocks_amplitude", "qem_masked_moments", "qem_polar_layout", "qem_decode_range",
+           "qem_pixel_classes", "qem_masked_sum_complement")
 
 
 class QemError(RuntimeError):
@@ -42,7 +43,7 @@ class QemError(RuntimeError):
 
 
 class MalformedStream(QemError, ValueError):
-    """A decoded stream failed a qem-pair-v1 check; the query has no result."""
+    """A decoded stream failed a qem-pair-v2 check; the query has no result."""
 
 
 class TaintedBaseline(QemError):
@@ -86,7 +87,10 @@ def lib() -> ctypes.CDLL:
         "qem_encode_append": ([vp, vp, i64, vp], ctypes.c_int),
         "qem_masked_sum": ([vp, vp, i32, i32, vp, ctypes.POINTER(i32), i32, vp], ctypes.c_int),
         "qem_masked_sum_delta": ([vp, vp, i32, i32, vp, ctypes.POINTER(i32), i32, vp], ctypes.c_int),
+        "qem_masked_sum_complement": ([vp, vp, i32, i32, vp, ctypes.POINTER(i32), i32, vp], ctypes.c_int),
         "qem_decode_blocks": ([vp, i64, i64, vp, i32, vp], ctypes.c_int),
+        "qem_decode_range": ([vp, i64, i64, vp, i32, vp], ctypes.c_int),
+        "qem_pixel_classes": ([vp, vp], ctypes.c_int),
         "qem_finish": ([vp, vp], ctypes.c_int),
         "qem_info": ([vp, ctypes.POINTER(Info)], ctypes.c_int),
         "qem_query_counters": ([vp, ctypes.POINTER(u64), ctypes.POINTER(u64), vp], ctypes.c_int),
@@ -247,6 +251,13 @@ class Resident:
         return self._query(lib().qem_masked_sum_delta, "qem_masked_sum_delta", mask, block_stride, out_bits,
                            out, wait, stream)
 
+    def masked_sum_complement(self, mask: torch.Tensor, block_stride: int = 1, out_bits: int = 0,
+                              out: torch.Tensor | None = None, wait: bool = True, stream=None) -> torch.Tensor:
+        """The same image as masked_sum, as the cached full-detector image minus the valid pixels
+        outside the mask (the cheaper route for dense masks such as a dark field)."""
+        return self._query(lib().qem_masked_sum_complement, "qem_masked_sum_complement", mask, block_stride,
+                           out_bits, out, wait, stream)
+
     def masked_sum_noalloc(self, mask: torch.Tensor, out: torch.Tensor, block_stride: int = 1,
                            out_bits: int = 0, stream=None) -> torch.Tensor:
         """Masked sum that allocates no device memory (qem_masked_sum_noalloc): for callers that
@@ -278,6 +289,22 @@ class Resident:
         _check(lib().qem_decode_blocks(self._h, first, n, _dev_ptr(out), 1 if wait else 0, _stream(stream)),
                "qem_decode_blocks")
         return out
+
+    def decode_range(self, first_scan: int, n_scans: int, out: torch.Tensor | None = None, wait: bool = True,
+                     stream=None) -> torch.Tensor:
+        """Counts of scans [first_scan, first_scan + n_scans) as [n_scans][pixels] (native dtype)."""
+        if out is None:
+            _, n_pixels, bits, _ = self._static()
+            out = torch.empty((n_scans, n_pixels), dtype=_count_dtype(bits),
+                              device=torch.device("cuda", torch.cuda.current_device()))
+        _check(lib().qem_decode_range(self._h, first_scan, n_scans, _dev_ptr(out), 1 if wait else 0,
+                                      _stream(stream)), "qem_decode_range")
+        return out
+
+    def frame(self, scan: int, out: torch.Tensor | None = None, wait: bool = True, stream=None) -> torch.Tensor:
+        """One diffraction pattern (scan index scan_row * scan_cols + scan_col) as [det_rows][det_cols]."""
+        i = self.info()
+        return self.decode_range(scan, 1, out, wait, stream).view(i["det_rows"], i["det_cols"])
 
     # ---- interaction index ----------------------------------------------------
     def build_index(self, center=None, stream=None):
@@ -317,6 +344,13 @@ class Resident:
         v = np.zeros(i["n_pixels"], np.uint8)
         _check(lib().qem_export_valid(self._h, v.ctypes.data), "qem_export_valid")
         return v
+
+    def pixel_classes(self) -> np.ndarray:
+        """uint8 [pixels]: 1 for light streams (empty, sparse, run-decoded), 0 for pair-by-pair ones."""
+        i = self.info()
+        c = np.zeros(i["n_pixels"], np.uint8)
+        _check(lib().qem_pixel_classes(self._h, c.ctypes.data), "qem_pixel_classes")
+        return c
 
     def index_desc(self):
         """uint32 [n_blocks][leaves + roots] storage descriptors (width code in bits 30-31)."""

@@ -96,6 +96,11 @@ struct qem_resident {
     std::vector<Arena> idx_arenas;
     uint64_t idx_bytes = 0;
     uint8_t *d_mom_mask = nullptr;              // scratch mask store of the moments plan
+    unsigned long long *d_total = nullptr;      // cached full-detector image [B][512] (complement queries)
+    uint8_t *d_tot_mask = nullptr;              // scratch mask store of its plan
+    bool total_ready = false;
+    void *noalloc_scratch = nullptr;            // allocation-free masked sum: fixed working array
+    uint32_t *noalloc_flags = nullptr;          // and its pinned status word (owned by noalloc.cu)
     DevStatus *d_status = nullptr;
     DevStatus *h_status = nullptr;              // pinned
     std::map<int, Baseline> baselines;
@@ -198,6 +203,8 @@ void release(qem_resident *r)
     cudaFree(r->d_idx_base);
     cudaFree(r->d_idx_items);
     cudaFree(r->d_mom_mask);
+    cudaFree(r->d_total);
+    cudaFree(r->d_tot_mask);
     for (auto &kv : r->baselines) {
         cudaFree(kv.second.d_mask);
         cudaFree(kv.second.d_img);
@@ -322,6 +329,14 @@ int make_resident(int64_t scan_rows, int64_t scan_cols, int32_t det_rows, int32_
         e = cudaStreamSynchronize(st);        // host staging above goes out of scope
     if (e != cudaSuccess)
         return fail(cuda_status(e));
+    // set-up of the allocation-free masked sum on this device (its working array
+    // and kernels are loaded here, when allocating is expected, not at its first call);
+    // a failure leaves that one entry point unavailable, not the resident
+    if (noalloc_setup(r->device, &r->noalloc_scratch, &r->noalloc_flags) != QEM_OK) {
+        r->noalloc_scratch = nullptr;
+        r->noalloc_flags = nullptr;
+        cudaGetLastError();
+    }
     *out = r;
     return QEM_OK;
 }
@@ -414,8 +429,44 @@ int report_errors(qem_resident *r, cudaStream_t st)
     return timed_out ? QEM_ERR_TIMEOUT : QEM_ERR_MALFORMED;
 }
 
+// The cached full-detector image of the complement queries: every valid
+// pixel's stream decoded once (plan over the validity map, no baseline
+// touched), [B][512] uint64.  Synchronous on first use; a malformed stream
+// leaves no cache.
+int compute_total(qem_resident *r, cudaStream_t st)
+{
+    if (r->total_ready)
+        return QEM_OK;
+    int rc;
+    if ((!r->d_total && (rc = dalloc(&r->d_total, static_cast<size_t>(r->B) * kScans * 8))) ||
+        (!r->d_tot_mask && (rc = dalloc(&r->d_tot_mask, static_cast<size_t>(r->P)))))
+        return rc;
+    uint32_t *count = r->d_count + 4 * r->count_pair;
+    uint32_t *count_next = r->d_count + 4 * (r->count_pair ^ 1);
+    rc = timed(r, QEM_K_PLAN, st, [&] {
+        return launch_plan(r->d_valid, r->d_valid, r->d_pclass, r->d_tot_mask, r->P, 0, r->d_list, count, count_next,
+                           r->d_total, nullptr, r->B * kScans, 8, st);
+    });
+    if (rc)
+        return rc;
+    r->count_pair ^= 1;
+    rc = timed(r, QEM_K_DECODE_REDUCE, st, [&] {
+        return launch_decode_reduce(r->view(), r->tables(), r->d_list, count, 1, r->B, r->d_total, 8, r->d_status,
+                                    r->n_sm, st);
+    });
+    if (rc)
+        return rc;
+    QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+    if ((rc = bounded_wait(st)))
+        return rc;
+    if (r->h_status->flags)
+        return report_errors(r, st);
+    r->total_ready = true;
+    return QEM_OK;
+}
+
 int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, void *d_out, int32_t *used,
-          int32_t wait, cudaStream_t st, bool delta)
+          int32_t wait, cudaStream_t st, bool delta, bool complement = false)
 {
     if (!r || !d_mask || !d_out || k < 1 || (reinterpret_cast<uintptr_t>(d_out) & 15u))
         return QEM_ERR_ARG;
@@ -447,19 +498,25 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         if (bl.state == kValid && bl.out_bits == bits)
             mode = 1;
     }
+    if (complement) {
+        int rc0 = compute_total(r, st);
+        if (rc0)
+            return rc0;
+        mode = 2;
+    }
     uint32_t *count = r->d_count + 4 * r->count_pair;
     uint32_t *count_next = r->d_count + 4 * (r->count_pair ^ 1);
     // The index plan serves full queries; a delta lists its changed pixels one by
     // one (a moving mask changes pixels along its edge, which rarely fill a whole
     // group, and the per-pixel plan is the shorter launch).
-    const bool use_index = r->has_index && mode == 0;
+    const bool use_index = r->has_index && mode == 0 && !complement;
     int rc = timed(r, QEM_K_PLAN, st, [&] {
         if (use_index)
             return launch_plan_index(d_mask, r->d_pclass, bl.d_mask, r->P, mode, r->d_idx_slots, r->d_idx_root_leaf0,
                                      r->idx_R, r->d_list, r->d_idx_items, count, count_next, d_out, bl.d_img,
                                      n_elems, bits / 8, st);
         return launch_plan(d_mask, r->d_valid, r->d_pclass, bl.d_mask, r->P, mode, r->d_list, count, count_next,
-                           d_out, bl.d_img, n_elems, bits / 8, st);
+                           d_out, bl.d_img, n_elems, bits / 8, st, r->d_total, k);
     });
     if (rc)
         return rc;
@@ -470,8 +527,10 @@ int query(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, v
         const IndexView ix = use_index ? IndexView{r->d_idx_desc, r->d_idx_base, r->d_idx_items, r->idx_L,
                                                       r->idx_L + r->idx_R}
                                           : IndexView{nullptr, nullptr, nullptr, 0, 0};
+        // the index plan may list pixels with a minus sign (a leaf's stored sums minus
+        // its unmasked pixels), so its queries take the signed decode
         return launch_decode_reduce(r->view(), r->tables(), r->d_list, count, k, rows, d_out, bits / 8,
-                                    r->d_status, r->n_sm, st, mode == 1, bl.d_img, ix);
+                                    r->d_status, r->n_sm, st, mode == 1, bl.d_img, ix, mode != 0 || use_index);
     });
     if (rc)
         return rc;
@@ -671,9 +730,27 @@ int build_index(qem_resident *r, double cr, double cc, cudaStream_t st)
 
 }  // namespace
 
+namespace qem {
+int bounded_stream_wait(cudaStream_t st)
+{
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t e = cudaStreamQuery(st);
+        if (e == cudaSuccess)
+            return QEM_OK;
+        if (e != cudaErrorNotReady)
+            return cuda_status(e);
+        const double dt = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+        if (dt > kWaitSeconds)
+            return QEM_ERR_TIMEOUT;
+        std::this_thread::sleep_for(std::chrono::microseconds(dt < 0.01 ? 2 : 200));
+    }
+}
+}  // namespace qem
+
 extern "C" {
 
-const char *qem_abi(void) { return "qem-pair-v1"; }
+const char *qem_abi(void) { return "qem-pair-v2"; }
 
 const char *qem_status_string(int s)
 {
@@ -783,6 +860,12 @@ int qem_masked_sum_delta(qem_resident *r, const uint8_t *d_mask, int32_t k, int3
     return query(r, d_mask, k, out_bits, d_out, used, wait, static_cast<cudaStream_t>(stream), true);
 }
 
+int qem_masked_sum_complement(qem_resident *r, const uint8_t *d_mask, int32_t k, int32_t out_bits, void *d_out,
+                              int32_t *used, int32_t wait, void *stream)
+{
+    return query(r, d_mask, k, out_bits, d_out, used, wait, static_cast<cudaStream_t>(stream), false, true);
+}
+
 int qem_decode_blocks(qem_resident *r, int64_t first, int64_t n, void *d_out, int32_t wait, void *stream)
 {
     if (!r || !d_out || first < 0 || n < 0 || first + n > r->B_done ||
@@ -793,6 +876,30 @@ int qem_decode_blocks(qem_resident *r, int64_t first, int64_t n, void *d_out, in
         return QEM_OK;
     int rc = timed(r, QEM_K_DECODE_BLOCKS, st, [&] {
         return launch_decode_blocks(r->view(), r->tables(), first, n, d_out, r->d_status, st);
+    });
+    if (rc)
+        return rc;
+    if (wait) {
+        QEM_CK(cudaMemcpyAsync(r->h_status, r->d_status, sizeof(DevStatus), cudaMemcpyDeviceToHost, st));
+        rc = bounded_wait(st);
+        if (rc)
+            return rc;
+        return report_errors(r, st);
+    }
+    return QEM_OK;
+}
+
+int qem_decode_range(qem_resident *r, int64_t first_scan, int64_t n_scans, void *d_out, int32_t wait, void *stream)
+{
+    if (!r || first_scan < 0 || n_scans < 0 || first_scan + n_scans > r->B_done * kScans)
+        return QEM_ERR_ARG;
+    if (n_scans == 0)
+        return QEM_OK;
+    if (!d_out || (reinterpret_cast<uintptr_t>(d_out) & static_cast<uintptr_t>(r->w - 1)))
+        return QEM_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = timed(r, QEM_K_DECODE_BLOCKS, st, [&] {
+        return launch_decode_range(r->view(), r->tables(), first_scan, n_scans, d_out, r->d_status, st);
     });
     if (rc)
         return rc;
@@ -902,6 +1009,8 @@ int qem_info(const qem_resident *r, qem_info_t *o)
     for (auto &kv : r->baselines)
         dev += r->P + static_cast<uint64_t>((r->B + kv.first - 1) / kv.first) * kScans * 8;
     dev += sizeof(HostTables);
+    if (r->d_total)
+        dev += static_cast<uint64_t>(r->B) * kScans * 8 + r->P;
     if (r->has_index)
         dev += r->idx_bytes + static_cast<uint64_t>(r->B) * (r->idx_L + r->idx_R) * 4 + r->B * 8 +
                static_cast<uint64_t>(r->idx_L) * 64 * 4 + (r->idx_R + 1) * 4 + (r->idx_L + r->idx_R) * 4;
@@ -1152,6 +1261,14 @@ int qem_index_desc(const qem_resident *r, uint32_t *h_desc)
     return QEM_OK;
 }
 
+int qem_pixel_classes(const qem_resident *r, uint8_t *h_class)
+{
+    if (!r || !h_class)
+        return QEM_ERR_ARG;
+    QEM_CK(cudaMemcpy(h_class, r->d_pclass, static_cast<size_t>(r->P), cudaMemcpyDeviceToHost));
+    return QEM_OK;
+}
+
 int qem_model_tables(uint16_t *h_freq, uint8_t *h_amax, uint32_t *h_cost)
 {
     const HostTables &T = host_tables();
@@ -1192,6 +1309,9 @@ int resident_query_view(const qem_resident *r, ResidentQuery *q)
     q->n_sm = r->n_sm;
     q->device = r->device;
     q->valid = r->d_valid;
+    q->pclass = r->d_pclass;
+    q->noalloc_scratch = r->noalloc_scratch;
+    q->noalloc_flags = r->noalloc_flags;
     return QEM_OK;
 }
 }  // namespace qem

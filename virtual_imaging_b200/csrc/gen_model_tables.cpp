@@ -1,5 +1,5 @@
 // gen_model_tables.cpp -- writes model_tables.inc, the frozen pair-model data
-// of the library's bitstream qem-pair-v1 (spec S4).
+// of the library's bitstream qem-pair-v2 (spec S4).
 //
 // Page "Paired-count resident layout", "Operation pipeline" step 2: streams
 // are coded with "a 1024-state tANS table from 32 Poisson pair models", and
@@ -99,7 +99,7 @@ Model make_model(int m)
 
 int main()
 {
-    std::printf("// model_tables.inc -- frozen pair-model data of qem-pair-v1 (spec S4).\n"
+    std::printf("// model_tables.inc -- frozen pair-model data of qem-pair-v2 (spec S4).\n"
                 "// Written by gen_model_tables.cpp; do not edit by hand.\n"
                 "// kFreq[m][a + 16 b]: tANS frequencies of pair (a, b), summing to 1024;\n"
                 "// kBox[m]: largest count the model codes; kCost[m][v]: selection cost of\n"

@@ -18,7 +18,7 @@
 //    optionally with their float32 square-root amplitude (k_amplitude).
 // Page "Backend Optimization Matrix", CoM/DPC rows: fused moment numerators
 // and denominator over the same decode (k_moments).
-// Bit-level choices follow the library's spec qem-pair-v1 (S1-S7).
+// Bit-level choices follow the library's spec qem-pair-v2 (S1-S7).
 //
 // No kernel traps or asserts: malformed input sets flags in DevStatus and the
 // affected lane contributes zeros.  Every loop ends: a fixed trip count, a
@@ -56,22 +56,27 @@ __device__ __forceinline__ void report(DevStatus *st, uint32_t flag)
 // returns false (the query then reports an error instead of a result).
 constexpr uint32_t kWaitLimit = 1u << 22;
 
-__device__ __forceinline__ void tables_start(uint64_t *bar, void *s_dst0, const void *g_src0, uint32_t bytes0,
-                                             void *s_dst1, const void *g_src1, uint32_t bytes1)
+__device__ __forceinline__ void tables_start(uint64_t *bar, uint32_t *s_dec, const uint32_t *dec_g,
+                                             const uint32_t *runs_g, int skip_count)
 {
+    // one 4 KB table per model at its model's place: the run-event tables of
+    // the models below skip_count, the decode tables of the others (two copies)
     const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes0 + bytes1) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(s_dst0))),
-                 "l"(g_src0), "r"(bytes0), "r"(b)
+    const uint32_t run_bytes = static_cast<uint32_t>(skip_count) * kStates * 4u;
+    const uint32_t dec_bytes = static_cast<uint32_t>(kModels - skip_count) * kStates * 4u;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(run_bytes + dec_bytes)
                  : "memory");
-    if (bytes1)
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + skip_count * kStates))),
+                 "l"(dec_g + skip_count * kStates), "r"(dec_bytes), "r"(b)
+                 : "memory");
+    if (run_bytes)
         asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                         static_cast<uint32_t>(__cvta_generic_to_shared(s_dst1))),
-                     "l"(g_src1), "r"(bytes1), "r"(b)
+                         static_cast<uint32_t>(__cvta_generic_to_shared(s_dec))),
+                     "l"(runs_g), "r"(run_bytes), "r"(b)
                      : "memory");
 }
 
@@ -164,7 +169,9 @@ struct Stream {
     int shift;
     uint32_t base;
     uint32_t c;          // constant value / sparse count
-    uint32_t x;          // tANS state minus 1024
+    uint32_t x;          // tANS state minus 1024 (state A: every pair, or the even pairs)
+    uint32_t x2;         // state B minus 1024 (odd pairs) when two
+    bool two;            // paired stream coded with two interleaved states (spec S3/S5)
     const uint8_t *s;
     uint32_t len;
     uint32_t tans_len;   // paired: bytes of the tANS section
@@ -300,6 +307,13 @@ __device__ bool open_stream(Stream &S, int w, DevStatus *st)
     if (S.bt.n < 10)
         S.bt.refill();
     S.x = S.bt.get(10);
+    S.two = S.model >= kOneStateModels;
+    S.x2 = 0;
+    if (S.two) {
+        if (S.bt.n < 10)
+            S.bt.refill();
+        S.x2 = S.bt.get(10);
+    }
     return true;
 }
 
@@ -307,7 +321,7 @@ __device__ bool open_stream(Stream &S, int w, DevStatus *st)
 // length exactly ceil(T/8), zero pad bits.
 __device__ bool close_paired(Stream &S, DevStatus *st)
 {
-    if (S.x != 0) {
+    if (S.x != 0 || S.x2 != 0) {
         report(st, kErrState);
         return false;
     }
@@ -343,6 +357,42 @@ __device__ __forceinline__ uint32_t tans_step(Stream &S, const uint32_t *dec)
 // table address is formed by mad (FMA pipe), the mask by bmsk, the new state
 // by one lop3 (newbase | (bits & mask); newbase's low nb bits are zero), the
 // reservoir shift by a funnel shift, the pair by prmt.
+// The same step in two halves, for two interleaved states: the table load
+// (which depends only on the state) and the bit consumption (which depends on
+// the reservoir, so state B's consumption follows state A's), so that both
+// states' loads are in flight together.
+__device__ __forceinline__ uint32_t tab_load(uint32_t x, uint32_t dec_sa)
+{
+    uint32_t e;
+    asm("{\n\t"
+        ".reg .b32 a;\n\t"
+        "mad.lo.u32 a, %1, 4, %2;\n\t"
+        "ld.shared.u32 %0, [a];\n\t"
+        "}"
+        : "=r"(e)
+        : "r"(x), "r"(dec_sa));
+    return e;
+}
+
+__device__ __forceinline__ uint32_t consume(uint32_t e, uint32_t &x, uint32_t &lo, uint32_t &hi, int &n)
+{
+    uint32_t pk, nb;
+    asm("{\n\t"
+        ".reg .b32 m, t;\n\t"
+        "bfe.u32 %1, %6, 10, 4;\n\t"
+        "bmsk.clamp.b32 m, 0, %1;\n\t"
+        "and.b32 t, %4, m;\n\t"
+        "lop3.b32 %3, %6, 1023, t, 0xEA;\n\t"
+        "shf.r.clamp.b32 %4, %4, %5, %1;\n\t"
+        "shr.b32 %5, %5, %1;\n\t"
+        "prmt.b32 %0, %6, 0, 0x4342;\n\t"
+        "}"
+        : "=r"(pk), "=r"(nb), "+r"(n), "+r"(x), "+r"(lo), "+r"(hi)
+        : "r"(e));
+    n -= static_cast<int>(nb);
+    return pk;
+}
+
 __device__ __forceinline__ uint32_t fast_step(uint32_t &x, uint32_t &lo, uint32_t &hi, int &n, uint32_t dec_sa)
 {
     uint32_t pk, nb;
@@ -378,7 +428,15 @@ __device__ __forceinline__ void paired_segment(Stream &S, const uint32_t *dec, u
             S.bt.refill();
         if (S.br.n < 2 * S.shift)
             S.br.refill();
-        const uint32_t ent = tans_step(S, dec);
+        // a segment starts at an even pair: odd jj is an odd pair, on state B
+        // when the stream has two states
+        uint32_t ent;
+        if ((jj & 1) && S.two) {
+            ent = dec[S.x2];
+            S.x2 = (ent & 1023u) | S.bt.get(static_cast<int>((ent >> 10) & 15u));
+        } else {
+            ent = tans_step(S, dec);
+        }
         const uint32_t lo = S.br.get(2 * S.shift);
         const uint32_t va = S.base + ((((ent >> 16) & 0xFFu) << S.shift) | (lo & mask));
         const uint32_t vb = S.base + (((ent >> 24) << S.shift) | ((lo >> S.shift) & mask));
@@ -537,10 +595,23 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
             int wi = kSlotWords - 1;
             uint64_t acc = 0;
             int nacc = 0;
-            uint32_t Tbits = 10;
-            uint32_t X = kStates;
+            // models 8-31 code pair j on state A (even j) or B (odd j); both start
+            // at 1024 after pair 255 (spec S3/S5)
+            const bool two = model >= kOneStateModels;
+            uint32_t Tbits = two ? 20u : 10u;
+            uint32_t XA = kStates, XB = kStates;
+            auto push = [&](uint32_t bits, uint32_t k) {
+                acc = (acc << k) | bits;
+                nacc += static_cast<int>(k);
+                if (nacc >= 32) {
+                    slot[wi--] = static_cast<uint32_t>(acc >> (nacc - 32));
+                    nacc -= 32;
+                }
+            };
             const T *q = col + static_cast<size_t>(kScans - 2) * P;
             for (int j = kPairs - 1; j >= 0; --j, q -= 2 * static_cast<size_t>(P)) {
+                const bool on_b = two && (j & 1);
+                uint32_t X = on_b ? XB : XA;
                 const uint32_t a = (static_cast<uint32_t>(q[0]) - base) >> shift;
                 const uint32_t bb = (static_cast<uint32_t>(q[P]) - base) >> shift;
                 const uint32_t es = __ldg(esym + a + 16u * bb);
@@ -551,20 +622,17 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
                 const uint32_t chunk = X & ((1u << k) - 1u);
                 const uint32_t y = X >> k;
                 X = kStates + __ldg(eslot + cum + (y - f));
-                acc = (acc << k) | chunk;
-                nacc += static_cast<int>(k);
+                if (on_b)
+                    XB = X;
+                else
+                    XA = X;
+                push(chunk, k);
                 Tbits += k;
-                if (nacc >= 32) {
-                    slot[wi--] = static_cast<uint32_t>(acc >> (nacc - 32));
-                    nacc -= 32;
-                }
             }
-            acc = (acc << 10) | (X - kStates);
-            nacc += 10;
-            if (nacc >= 32) {
-                slot[wi--] = static_cast<uint32_t>(acc >> (nacc - 32));
-                nacc -= 32;
-            }
+            // the section starts with x_A, then x_B: prepended last, in reverse
+            if (two)
+                push(XB - kStates, 10u);
+            push(XA - kStates, 10u);
             if (nacc > 0)
                 slot[wi] = static_cast<uint32_t>(acc << (32 - nacc));
             {
@@ -913,11 +981,13 @@ constexpr int kPlanThreads = 256;
 // front (count[0]), light ones (empty, sparse, run-decoded) from the back
 // (count[1], list[P-1], list[P-2], ...), so that warps meet one kind of work.
 // Order inside a class does not matter to the sums (integer addition).
-// Full query: mask && valid; delta: pixels whose (mask && valid) changed
-// against the stored baseline mask, leaving pixels flagged in bit 31.  Every
+// Full query (mode 0): mask && valid; delta (1): pixels whose (mask && valid)
+// changed against the stored baseline mask, leaving pixels flagged in bit 31;
+// complement (2): the valid pixels outside the mask, all flagged.  Every
 // thread then stores the new mask as the baseline.  Blocks past n_list_blocks initialise
 // the rows: a full query zeroes the output and the kept image, a delta starts
-// the output from the kept image (the decode adds its terms to both).  The
+// the output from the kept image, a complement query starts both from the
+// cached full-detector image (the decode adds its terms to both).  The
 // counter pair of the next query (count_next) is cleared here, so that no
 // separate clear is needed between queries.
 __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict__ mask,
@@ -927,7 +997,9 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
                                                       int n_list_blocks, uint32_t *__restrict__ list,
                                                       uint32_t *__restrict__ count,
                                                       uint32_t *__restrict__ count_next, uint4 *__restrict__ out,
-                                                      uint4 *__restrict__ keep, long long n_vec)
+                                                      uint4 *__restrict__ keep, long long n_vec,
+                                                      const unsigned long long *__restrict__ total, int stride,
+                                                      int out_bytes)
 {
     // the decode that follows may start its prologue (table copy) now; it
     // waits for this grid's completion before it reads anything written here
@@ -950,9 +1022,13 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
             if (mode == 0) {
                 emit = nw;
                 entry = static_cast<uint32_t>(p);
-            } else {
+            } else if (mode == 1) {
                 emit = nw != od;
                 entry = static_cast<uint32_t>(p) | (od ? 0x80000000u : 0u);
+            } else {
+                // complement: the valid pixels outside the mask, subtracted
+                emit = ok && mk == 0;
+                entry = static_cast<uint32_t>(p) | 0x80000000u;
             }
             light = pclass[p] != 0;
             base_mask[p] = mk;
@@ -985,14 +1061,30 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
             list[P - 1 - (s_at[1] + s_l[warp] + __popc(bl & below))] = entry;
         return;
     }
-    const long long stride = static_cast<long long>(gridDim.x - n_list_blocks) * blockDim.x;
+    const long long step = static_cast<long long>(gridDim.x - n_list_blocks) * blockDim.x;
     for (long long i = static_cast<long long>(blockIdx.x - n_list_blocks) * blockDim.x + threadIdx.x; i < n_vec;
-         i += stride) {
+         i += step) {
         if (mode == 0) {
             out[i] = make_uint4(0u, 0u, 0u, 0u);
-            keep[i] = make_uint4(0u, 0u, 0u, 0u);
-        } else {
+            if (keep)
+                keep[i] = make_uint4(0u, 0u, 0u, 0u);
+        } else if (mode == 1) {
             out[i] = keep[i];
+        } else {
+            // complement: every row starts from the cached full-detector image of
+            // its block (total is [B][512] uint64; row r holds block r * stride)
+            const long long per = 16 / out_bytes;
+            const long long e0 = i * per, row = e0 / kScans, col = e0 - row * kScans;
+            const unsigned long long *t = total + (row * stride) * kScans + col;
+            uint4 v;
+            if (out_bytes == 4)
+                v = make_uint4(static_cast<uint32_t>(t[0]), static_cast<uint32_t>(t[1]), static_cast<uint32_t>(t[2]),
+                               static_cast<uint32_t>(t[3]));
+            else
+                v = make_uint4(static_cast<uint32_t>(t[0]), static_cast<uint32_t>(t[0] >> 32),
+                               static_cast<uint32_t>(t[1]), static_cast<uint32_t>(t[1] >> 32));
+            out[i] = v;
+            keep[i] = v;
         }
     }
 }
@@ -1009,7 +1101,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(const uint8_t *__restrict
 // at a time and reduces them across the warp with redux.sync into the row's
 // shared slot; the warp that finishes a row piece's last task adds the slot to
 // the output with one global atomic per nonzero scan sum.
-template <int W, bool DELTA>
+template <int W, bool DELTA, bool ROOMY = false>
 __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec, const uint32_t *dec_g,
                                             uint32_t skip_models, const uint32_t *list, uint32_t n,
                                             uint32_t n_l, int tile,
@@ -1041,6 +1133,8 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     S.base = 0;
     S.c = 0;
     S.x = 0;
+    S.x2 = 0;
+    S.two = false;
     S.len = 0;
     bool ok = listed;
     if (ok)
@@ -1073,7 +1167,24 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     const bool runs = S.form == kPaired && S.shift == 0 && S.base == 0u && run_model;
     const uint32_t *dec = (run_model ? dec_g : s_dec) + S.model * kStates;
     const bool dense_lane = (S.form == kPaired && !runs) || S.form == kLiteral || S.form == kConstant;
-    const bool fast = S.form == kPaired && !runs && S.shift == 0 && S.base == 0u;
+    // A warp with a paired lane that needs the general step (a base or raw
+    // low bits: one count of 16 or more in a low-count stream is enough) runs
+    // the general step on all its paired lanes: with both kinds in one warp
+    // the fast loop and the general loop would run one after the other.
+    const bool plain_warp = __all_sync(kFull, !(S.form == kPaired && !runs) || (S.shift == 0 && S.base == 0u));
+    // uint8: a warp whose pair-by-pair lanes all use two-state models takes the
+    // two-state loop even when some lanes carry a base or raw low bits (one
+    // count of 16 or more in a low-count stream is enough): those are added
+    // per pair after the table steps (8-bit values keep the packed halves apart)
+    // (kernels launched with room for more registers per thread only)
+    const bool two_lane = S.form == kPaired && !runs && S.two;
+    bool fast = plain_warp && two_lane && S.shift == 0 && S.base == 0u;
+    bool raw_warp = false;
+    if constexpr (W == 1 && ROOMY) {
+        const bool all_two = __all_sync(kFull, !(S.form == kPaired && !runs) || S.two);
+        raw_warp = __any_sync(kFull, two_lane && (S.shift != 0 || S.base != 0u));
+        fast = all_two && two_lane;
+    }
     uint32_t over = 0;
     // warps whose lanes hold only empty, sparse or run-decoded streams skip the per-scan loop
     const bool dense = __any_sync(kFull, dense_lane);
@@ -1094,12 +1205,35 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
         for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
             uint32_t pk[16];
             if (fast) {
+                // two interleaved states (fast streams use models 8-31, spec S3):
+                // both table loads first, then the bits of pair A, then pair B
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    // top-ups before steps 0, 3, 6, 9, 12, 15: <= 30 bits per 3 steps
+                for (int jj = 0; jj < 16; jj += 2) {
+                    const uint32_t ea = tab_load(S.x, dec_sa);
+                    const uint32_t eb = tab_load(S.x2, dec_sa);
+                    // top-ups before pairs 0, 3, 6, 9, 12, 15: <= 30 bits per 3 pairs
                     if (jj % 3 == 0 && S.bt.n < 30)
                         S.bt.refill();
-                    pk[jj] = fast_step(S.x, S.bt.lo, S.bt.hi, S.bt.n, dec_sa);
+                    pk[jj] = consume(ea, S.x, S.bt.lo, S.bt.hi, S.bt.n);
+                    if ((jj + 1) % 3 == 0 && S.bt.n < 30)
+                        S.bt.refill();
+                    pk[jj + 1] = consume(eb, S.x2, S.bt.lo, S.bt.hi, S.bt.n);
+                }
+                if constexpr (W == 1 && ROOMY) {
+                  if (raw_warp) {
+                    // v = base + (hi << shift | lo), both halves at once
+                    const uint32_t m = (1u << S.shift) - 1u;
+                    const uint32_t bpk = S.base | (S.base << 16);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        if (S.br.n < 2 * S.shift)
+                            S.br.refill();
+                        const uint32_t lo = S.br.get(2 * S.shift);
+                        const uint32_t v = ((pk[jj] << S.shift) | (lo & m) | (((lo >> S.shift) & m) << 16)) + bpk;
+                        over |= (v & 0xFFFFu) | (v >> 16);
+                        pk[jj] = v;
+                    }
+                  }
                 }
             } else if (S.form == kPaired && !runs) {
                 uint32_t vv[32];
@@ -1333,9 +1467,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     uint32_t *s_acc = s_stage + MAXW * 16;
     __shared__ __align__(8) uint64_t s_bar;
     if (threadIdx.x == 0)
-        tables_start(&s_bar, s_dec + skip_count * kStates, dec_g + skip_count * kStates,
-                     static_cast<uint32_t>(kModels - skip_count) * kStates * 4u, s_dec, runs_g,
-                     static_cast<uint32_t>(skip_count) * kStates * 4u);
+        tables_start(&s_bar, s_dec, dec_g, runs_g, skip_count);
     bool ready = false;
     // per-CTA counters (rows, streams), added to the status once at the end
     __shared__ uint32_t s_cnt[2];
@@ -1434,9 +1566,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
             }
         }
         ok = __shfl_sync(kFull, ok, 0);
-        if (ok)
-            decode_task<W, DELTA>(v, s_dec, dec_g, skip_models, list, n, n_l, tile, row * stride,
-                                  s_acc + slot * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready, lane, st);
+        // a wait that ran out leaves the slot to its owner: this warp neither
+        // decodes nor counts the task (the query reports QEM_ERR_TIMEOUT), so
+        // no other piece's sums are flushed into this row
+        if (!ok)
+            continue;
+        decode_task<W, DELTA, (THREADS <= 512 && DELTA)>(v, s_dec, dec_g, skip_models, list, n, n_l, tile, row * stride,
+                              s_acc + slot * kScans, s_stage + warp * 16, s_cnt, &s_bar, ready, lane, st);
         // this warp's slot additions happen before its count
         __threadfence_block();
         __syncwarp();
@@ -1555,6 +1691,8 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
             S.base = 0;
             S.c = 0;
             S.x = 0;
+            S.x2 = 0;
+            S.two = false;
             S.len = 0;
             bool ok = listed;
             if (ok)
@@ -1731,6 +1869,8 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
         S.base = 0;
         S.c = 0;
         S.x = 0;
+        S.x2 = 0;
+        S.two = false;
         S.len = 0;
         bool ok = v.valid[p] != 0;
         if (ok)
@@ -1796,6 +1936,122 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
                 dst[i * P] = c;
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// a7b: scan-range decode (frames)
+// ---------------------------------------------------------------------------
+// Scans [first, first + n) in native frames: one thread per stream of every
+// block the range touches; a stream is decoded only up to the last pair the
+// range needs and its counts inside the range are stored down its pixel
+// column of out[n][P] (coalesced per scan, as in the block decode).  Literal
+// counts are read directly at their byte offset.  Because paired streams
+// stop early, their end-of-stream state is not checked here (block decodes
+// and queries check it); everything that is read is checked (header, fields,
+// form lengths, sparse order, value range, and that no read passes the
+// stream's extent).  Invalid pixels come out 0.
+template <int W>
+__global__ void __launch_bounds__(256) k_decode_range(View v, const uint32_t *__restrict__ dec_g,
+                                                     long long first, long long n, void *__restrict__ out,
+                                                     DevStatus *__restrict__ st)
+{
+    using T = typename std::conditional<W == 1, uint8_t, uint16_t>::type;
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *s_dec = smem;
+    __shared__ __align__(8) uint64_t s_bar;
+    if (threadIdx.x == 0)
+        tables_start(&s_bar, s_dec, dec_g, dec_g, 0);
+    __syncthreads();
+    bool ready = false;
+    T *o = reinterpret_cast<T *>(out);
+    const long long b0 = first / kScans, b1 = (first + n - 1) / kScans;
+    const long long total = (b1 - b0 + 1) * v.P;
+    const size_t P = static_cast<size_t>(v.P);
+    for (long long sid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; sid < total;
+         sid += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long bi = sid / v.P;
+        const int p = static_cast<int>(sid - bi * v.P);
+        const long long b = b0 + bi;
+        // this block's scans inside the range: [lo, hi) of its 512
+        const int lo = static_cast<int>(max(first, b * kScans) - b * kScans);
+        const int hi = static_cast<int>(min(first + n, (b + 1) * kScans) - b * kScans);
+        T *dst = o + (static_cast<size_t>(b * kScans + lo - first)) * P + p;   // row of scan lo
+        Stream S;
+        S.form = kEmpty;
+        S.model = 0;
+        S.shift = 0;
+        S.base = 0;
+        S.c = 0;
+        S.x = 0;
+        S.x2 = 0;
+        S.two = false;
+        S.len = 0;
+        bool ok = v.valid[p] != 0;
+        if (ok)
+            ok = locate(v, b, p, S.s, S.len, st);
+        if (ok)
+            ok = open_stream(S, W, st);
+        if (!ok)
+            S.form = kEmpty;
+        if (S.form == kPaired) {
+            if (!ready) {
+                if (!tables_wait(&s_bar, st))
+                    S.form = kEmpty;
+                ready = true;
+            }
+        }
+        if (S.form == kPaired) {
+            const uint32_t *dec = s_dec + S.model * kStates;
+            uint32_t over = 0;
+            const int last_seg = (hi - 1) >> 5;
+            for (int seg = 0; seg <= last_seg; ++seg) {
+                uint32_t vv[32];
+                paired_segment(S, dec, vv, over);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int sc = seg * 32 + i;
+                    if (sc >= lo && sc < hi)
+                        dst[(sc - lo) * P] = static_cast<T>(vv[i]);
+                }
+            }
+            if (over > (W == 1 ? 0xFFu : 0xFFFFu))
+                report(st, kErrValue);
+            if (S.bt.consumed() > 8ll * S.tans_len || S.br.consumed() > 8ll * 64 * S.shift)
+                report(st, kErrLength);
+        } else if (S.form == kLiteral) {
+            for (int sc = lo; sc < hi; ++sc)
+                dst[(sc - lo) * P] = static_cast<T>(load_native(S.s + 2 + sc * W, W));
+        } else if (S.form == kSparse) {
+            for (int sc = lo; sc < hi; ++sc)
+                dst[(sc - lo) * P] = 0;
+            int prev = -1;
+            for (uint32_t k = 0; k < S.c; ++k) {
+                if (S.bt.n < 9)
+                    S.bt.refill();
+                const int pos = static_cast<int>(S.bt.get(9));
+                if (S.br.n < 16)
+                    S.br.refill();
+                const uint32_t val = S.br.get(8 * W);
+                if (pos <= prev || val == 0u) {
+                    report(st, kErrSparse);
+                    break;
+                }
+                if (pos >= hi)
+                    break;
+                if (pos >= lo)
+                    dst[(pos - lo) * P] = static_cast<T>(val);
+                prev = pos;
+            }
+        } else {
+            const T c = static_cast<T>(S.form == kConstant ? S.c : 0u);
+            for (int sc = lo; sc < hi; ++sc)
+                dst[(sc - lo) * P] = c;
+        }
+    }
+    __syncthreads();
+    // a CTA leaves only after its table copy has landed
+    if (threadIdx.x == 0)
+        tables_wait(&s_bar, st);
 }
 
 // float32 square-root amplitude of decoded counts (the feed's second output;
@@ -1870,9 +2126,7 @@ __global__ void __launch_bounds__(768, 1) k_index_sums(View v, const uint32_t *_
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ uint32_t s_cnt[2];
     if (threadIdx.x == 0)
-        tables_start(&s_bar, s_dec + skip_count * kStates, dec_g + skip_count * kStates,
-                     static_cast<uint32_t>(kModels - skip_count) * kStates * 4u, s_dec, runs_g,
-                     static_cast<uint32_t>(skip_count) * kStates * 4u);
+        tables_start(&s_bar, s_dec, dec_g, runs_g, skip_count);
     if (threadIdx.x < 2)
         s_cnt[threadIdx.x] = 0u;
     __syncthreads();
@@ -1967,8 +2221,14 @@ __global__ void __launch_bounds__(512) k_index_pack(const uint32_t *__restrict__
 // A leaf whose every pixel is in the mask (full query), or whose every pixel
 // enters, or every pixel leaves, the mask (delta) becomes one index item; a
 // root whose leaves all do so in the same direction becomes one root item
-// instead.  The remaining masked (changed) pixels go to the residual list as
-// in k_plan.  The counts are count[0] heavy, count[1] light, count[2] items.
+// instead.  In a full query, a leaf partly in the mask becomes an item plus
+// its unmasked pixels with a minus sign when their decode costs less than
+// the masked pixels' (planner weights: a pair-by-pair stream kPlanHeavy, a
+// light one kPlanLight, an item kPlanItem).  The remaining masked (changed)
+// pixels go to the residual list as in k_plan.  The counts are count[0]
+// heavy, count[1] light, count[2] items.  Entries with bit 31 set subtract,
+// so the decode that follows is the signed (delta) instantiation.
+constexpr uint32_t kPlanHeavy = 16, kPlanLight = 1, kPlanItem = 2;
 __global__ void __launch_bounds__(512) k_plan_index(const uint8_t *__restrict__ mask,
                                                    const uint8_t *__restrict__ pclass,
                                                    uint8_t *__restrict__ base_mask, int P, int mode,
@@ -1983,7 +2243,8 @@ __global__ void __launch_bounds__(512) k_plan_index(const uint8_t *__restrict__ 
         count_next[threadIdx.x] = 0u;
     if (static_cast<int>(blockIdx.x) < R) {
         constexpr int NW = 16;
-        __shared__ int s_state[NW];            // per leaf: 1 all enter/in, 2 all leave, 0 otherwise, -1 none
+        __shared__ int s_state[NW];            // per leaf: 1 all enter/in, 2 all leave, 3 item minus
+                                               // unmasked pixels, 0 otherwise, -1 none
         __shared__ uint32_t s_h[NW], s_l[NW], s_at[2];
         const int r = blockIdx.x;
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -2021,16 +2282,42 @@ __global__ void __launch_bounds__(512) k_plan_index(const uint8_t *__restrict__ 
             all_in = __all_sync(kFull, all_in);
             all_out = __all_sync(kFull, all_out) && mode == 1;
             state = all_in ? 1 : (all_out ? 2 : 0);
+            if (mode == 0) {
+                // planner: decode the leaf's masked pixels, or take its stored sums
+                // and subtract its unmasked pixels, whichever decodes less (cost of
+                // a stream by its class; an item reads 512 stored sums)
+                uint32_t c_in = 0, c_out = 0;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const uint32_t p = k ? pp.y : pp.x;
+                    const uint32_t c = light[k] ? kPlanLight : kPlanHeavy;
+                    if (p < static_cast<uint32_t>(P)) {
+                        c_in += emit[k] ? c : 0u;
+                        c_out += emit[k] ? 0u : c;
+                    }
+                }
+                c_in = __reduce_add_sync(kFull, c_in);
+                c_out = __reduce_add_sync(kFull, c_out);
+                if (state == 0 && kPlanItem + c_out < c_in) {
+                    state = 3;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const uint32_t p = k ? pp.y : pp.x;
+                        emit[k] = p < static_cast<uint32_t>(P) && !emit[k];
+                        entry[k] = p | 0x80000000u;
+                    }
+                }
+            }
         }
         if (lane == 0)
             s_state[warp] = state;
         __syncthreads();
-        // the root as one item when all its leaves go the same way
+        // the root as one item when all its leaves are wholly in (or wholly leave)
         int rs = s_state[0];
         for (int k = 1; k < nl; ++k)
             rs = s_state[k] == rs ? rs : 0;
-        const bool root_item = nl > 0 && rs > 0;
-        if (state > 0 || root_item) {
+        const bool root_item = nl > 0 && (rs == 1 || rs == 2);
+        if (state == 1 || state == 2 || root_item) {
             emit[0] = emit[1] = false;        // covered by an index item
         }
         // index items: one reservation per CTA (the root, or its whole leaves in order)
@@ -2162,7 +2449,8 @@ cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const
 
 cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t *pclass, uint8_t *base_mask,
                         int P, int mode, uint32_t *list, uint32_t *count, uint32_t *count_next, void *out,
-                        void *keep, long long n_elems, int out_bytes, cudaStream_t st)
+                        void *keep, long long n_elems, int out_bytes, cudaStream_t st,
+                        const unsigned long long *total, int stride)
 {
     const long long n_vec = n_elems * out_bytes / 16;
     const int n_list = (P + kPlanThreads - 1) / kPlanThreads;
@@ -2170,7 +2458,7 @@ cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t
     fill = fill < 1 ? 1 : (fill > 8 * sm_count() ? 8 * sm_count() : fill);
     k_plan<<<n_list + fill, kPlanThreads, 0, st>>>(mask, valid, pclass, base_mask, P, mode, n_list, list, count,
                                                    count_next, static_cast<uint4 *>(out), static_cast<uint4 *>(keep),
-                                                   n_vec);
+                                                   n_vec, total, stride, out_bytes);
     return cudaGetLastError();
 }
 
@@ -2203,21 +2491,44 @@ cudaError_t launch_dr(View v, Tables tb, const uint32_t *list, const uint32_t *c
                               list, count, stride, rows, out, keep, out_bytes, ix, status);
 }
 
+cudaError_t preload_query_kernels()
+{
+    const void *fns[] = {reinterpret_cast<const void *>(k_decode_reduce<1, 768, false>),
+                         reinterpret_cast<const void *>(k_decode_reduce<2, 512, false>)};
+    const size_t smem[] = {kTableBytes + 768 / 32 * 16 * sizeof(uint32_t) + kMaxSlots * kScans * sizeof(uint32_t),
+                           kTableBytes + 512 / 32 * 16 * sizeof(uint32_t) + kMaxSlots * kScans * sizeof(uint32_t)};
+    for (int i = 0; i < 2; ++i) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, fns[i]);
+        if (e == cudaSuccess)
+            e = ensure_smem(fns[i], smem[i]);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count, int stride,
                                  long long rows, void *out, int out_bytes, DevStatus *status, int n_sm,
-                                 cudaStream_t st, bool delta, void *keep, IndexView ix)
+                                 cudaStream_t st, bool delta, void *keep, IndexView ix, bool signed_list)
 {
     // u8 deltas (few tasks, each warp's decode latency is the critical path)
-    // run at 512 threads, with room for more registers; full queries at 768
-    if (v.w == 1)
-        return delta ? launch_dr<1, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
-                                               n_sm, st)
-                     : launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status,
-                                                n_sm, st);
-    return delta ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
-                                           st)
-                 : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
-                                            st);
+    // run at 512 threads, with room for more registers; full queries at 768,
+    // or 640 when their list has subtracted entries (index plans, complement):
+    // the signed decode needs a few more registers than 768 threads leave
+    if (v.w == 1) {
+        if (delta)
+            return launch_dr<1, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
+                                           st);
+        if (signed_list)
+            return launch_dr<1, 640, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
+                                           st);
+        return launch_dr<1, 768, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm, st);
+    }
+    return (delta || signed_list)
+               ? launch_dr<2, 512, true>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm, st)
+               : launch_dr<2, 512, false>(v, tb, list, count, stride, rows, out, keep, out_bytes, ix, status, n_sm,
+                                          st);
 }
 
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,
@@ -2233,6 +2544,24 @@ cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n
         k_decode_blocks<1><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
     else
         k_decode_blocks<2><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_range(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,
+                                cudaStream_t st)
+{
+    const size_t smem = kTableBytes;
+    const cudaError_t e = v.w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_decode_range<1>), smem)
+                                   : ensure_smem(reinterpret_cast<const void *>(k_decode_range<2>), smem);
+    if (e != cudaSuccess)
+        return e;
+    const long long blocks = (first + n - 1) / kScans - first / kScans + 1;
+    long long grid = (blocks * v.P + 255) / 256;
+    grid = grid < 1 ? 1 : (grid > 4ll * sm_count() ? 4ll * sm_count() : grid);
+    if (v.w == 1)
+        k_decode_range<1><<<static_cast<int>(grid), 256, smem, st>>>(v, tb.dec, first, n, out, status);
+    else
+        k_decode_range<2><<<static_cast<int>(grid), 256, smem, st>>>(v, tb.dec, first, n, out, status);
     return cudaGetLastError();
 }
 
@@ -2277,11 +2606,11 @@ cudaError_t launch_index_sums(View v, Tables tb, const uint32_t *slots, int L, l
     if (e != cudaSuccess)
         return e;
     if (v.w == 1)
-        k_index_sums<1><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, slots, L, b0, nblk,
-                                                  leafsum, status);
+        k_index_sums<1><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                                                  slots, L, b0, nblk, leafsum, status);
     else
-        k_index_sums<2><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count, slots, L, b0, nblk,
-                                                  leafsum, status);
+        k_index_sums<2><<<n_sm, 768, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                                                  slots, L, b0, nblk, leafsum, status);
     return cudaGetLastError();
 }
 

@@ -1,6 +1,6 @@
 // qem_internal.h -- shared declarations of libqem's host code and kernels.
 //
-// Bitstream: qem-pair-v1 (page "Paired-count resident layout", "Operation
+// Bitstream: qem-pair-v2 (page "Paired-count resident layout", "Operation
 // pipeline" step 2 and "Contract"; the bit-level choices are the library's
 // own written spec, sections S1-S7, cited as "spec Sn").
 #pragma once
@@ -20,6 +20,8 @@ constexpr int kGroupWords = 17;    // 1 x u32 base + 32 x u16 relative ends (spe
 constexpr int kSlotWords = 84;     // per-stream tANS scratch: >= ceil((10 + 256*10)/32) + 1 words, 16-byte multiple
 constexpr int kArenaPad = 64;      // zero bytes after the last block of an arena
 constexpr int kRunModels = 8;      // models that may be decoded by runs (their tables replace the decode tables in shared memory)
+constexpr int kOneStateModels = 8; // spec S3/S5: models 0-7 code a paired stream with one tANS state,
+                                   // models 8-31 with two interleaved ones (A: even pairs, B: odd pairs)
 
 enum Form : int { kEmpty = 0, kConstant = 1, kSparse = 2, kPaired = 3, kLiteral = 4 };
 
@@ -114,8 +116,25 @@ struct ResidentQuery {
     int n_sm;
     int device;
     const uint8_t *valid;
+    const uint8_t *pclass;        // per pixel: 1 = light streams, 0 = heavy
+    void *noalloc_scratch;        // device address of the fixed working array (noalloc.cu)
+    uint32_t *noalloc_flags;      // pinned host word for its status read-back
 };
 int resident_query_view(const qem_resident *r, ResidentQuery *q);
+
+// Set-up of the allocation-free masked sum on the current device, run when a
+// resident is created (noalloc.cu): looks up the fixed array's device address,
+// loads the kernels that call uses, and keeps one pinned host word per device
+// for its status.  QEM_OK or QEM_ERR_CUDA / QEM_ERR_OOM.
+int noalloc_setup(int device, void **scratch, uint32_t **h_flags);
+
+// Wait (bounded, ~60 s) until all work queued on `st` has finished, polling the
+// stream itself (creates nothing).  QEM_OK, QEM_ERR_TIMEOUT or QEM_ERR_CUDA.
+int bounded_stream_wait(cudaStream_t st);
+
+// Load the decode kernels a masked sum launches (lazy module loading would
+// otherwise load them at their first launch) and set their shared-memory limits.
+cudaError_t preload_query_kernels();
 
 // ---- kernel launchers (kernels.cu); all stream-ordered, return cudaError_t ----
 cudaError_t launch_generate(void *out, int bits, uint64_t seed, int64_t scan0, int64_t n_scans,
@@ -137,16 +156,20 @@ cudaError_t launch_enc_compact(const void *counts, int w, int P, int nblk, const
 // light class from the back (count[1]), clears count_next (the pair the next
 // query uses) and initialises the rows: mode 0 = full query (out = keep = 0),
 // 1 = delta (out = keep, the stride's kept image)
+// 2 = complement (the valid pixels outside the mask, subtracted; out = keep =
+// the rows r * stride of total, the cached full-detector image [B][512] uint64);
+// keep may be null in mode 0
 cudaError_t launch_plan(const uint8_t *mask, const uint8_t *valid, const uint8_t *pclass,
                         uint8_t *base_mask, int P, int mode, uint32_t *list, uint32_t *count,
                         uint32_t *count_next, void *out, void *keep, long long n_elems, int out_bytes,
-                        cudaStream_t st);
+                        cudaStream_t st, const unsigned long long *total = nullptr, int stride = 1);
 // keep (may be null): a second image that receives the same additions as out;
 // ix.desc null: no index items (count[2] is not read)
 cudaError_t launch_decode_reduce(View v, Tables tb, const uint32_t *list, const uint32_t *count,
                                  int stride, long long rows, void *out, int out_bytes,
                                  DevStatus *status, int n_sm, cudaStream_t st, bool delta = false,
-                                 void *keep = nullptr, IndexView ix = IndexView{nullptr, nullptr, nullptr, 0, 0});
+                                 void *keep = nullptr, IndexView ix = IndexView{nullptr, nullptr, nullptr, 0, 0},
+                                 bool signed_list = false);
 cudaError_t launch_amplitude(const void *counts, int w, float *amp, long long n, cudaStream_t st);
 // masked moments: out int64 [3][rows][512] = (sum x*wr, sum x*wc, sum x) per scan
 cudaError_t launch_moments(View v, Tables tb, const uint32_t *list, const uint32_t *count, const int32_t *weights,
@@ -165,5 +188,8 @@ cudaError_t launch_plan_index(const uint8_t *mask, const uint8_t *pclass, uint8_
                               int out_bytes, cudaStream_t st);
 cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n, void *out,
                                  DevStatus *status, cudaStream_t st);
+// scans [first, first + n) of the acquisition into out [n][P] (native dtype)
+cudaError_t launch_decode_range(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,
+                                cudaStream_t st);
 
 }  // namespace qem
