@@ -20,7 +20,8 @@ using namespace qem;
 namespace {
 
 constexpr size_t kArenaMax = size_t(1) << 30;       // payload allocation unit
-constexpr size_t kBatchRawBytes = size_t(64) << 20; // raw counts encoded per batch (L2-sized)
+constexpr size_t kBatchRawBytes = size_t(512) << 20; // raw counts encoded per batch (one host
+                                                      // synchronisation each, for the block placement)
 constexpr double kWaitSeconds = 60.0;
 
 enum BaseState { kNone = 0, kValid = 1, kTainted = 2 };

@@ -525,11 +525,18 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
 
         uint32_t nnz = 0, mn = 0xFFFFFFFFu, mx = 0;
         uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;      // first four nonzeros: scan | value << 16
+        // the histogram of the counts below 16 is taken in the same pass: when no
+        // count reaches 16 it is the hi histogram after the base (no shift)
+#pragma unroll
+        for (int v = 0; v < 16; ++v)
+            s_hist[v][tid] = 0;
         {
             const T *q = col;
 #pragma unroll 8
             for (int i = 0; i < kScans; ++i, q += P) {
                 const uint32_t v = *q;
+                if (v < 16u)
+                    s_hist[v][tid] += 1;
                 if (v && nnz < 4u) {
                     const uint32_t e = static_cast<uint32_t>(i) | (v << 16);
                     c0 = nnz == 0u ? e : c0;
@@ -559,20 +566,22 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
             const int span_bits = 32 - __clz(static_cast<int>(mx - base));
             const int shift = span_bits > 4 ? span_bits - 4 : 0;
 
+            const bool small = mx < 16u;             // every hi = count - base
+            if (!small) {
 #pragma unroll
-            for (int v = 0; v < 16; ++v)
-                s_hist[v][tid] = 0;
-            {
+                for (int v = 0; v < 16; ++v)
+                    s_hist[v][tid] = 0;
                 const T *q = col;
 #pragma unroll 8
                 for (int i = 0; i < kScans; ++i, q += P)
                     s_hist[(static_cast<uint32_t>(*q) - base) >> shift][tid] += 1;
             }
             const uint32_t maxhi = (mx - base) >> shift;
+            const uint32_t hoff = small ? base : 0u;
             uint32_t h[16];
 #pragma unroll
             for (int v = 0; v < 16; ++v)
-                h[v] = s_hist[v][tid];
+                h[v] = v + hoff < 16u ? s_hist[v + hoff][tid] : 0u;
             uint32_t best = 0xFFFFFFFFu;
             model = kModels - 1;
             for (int m = 0; m < kModels; ++m) {
