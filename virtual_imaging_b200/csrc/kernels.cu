@@ -833,9 +833,27 @@ __global__ void __launch_bounds__(kLayoutThreads) k_enc_layout(uint4 *__restrict
     }
 }
 
-// Write one stream's bytes (header and form payload, spec S2/S3) at o.
+// Counts of scans i0 .. i0 + kColBatch - 1 of one pixel column (stride P):
+// the loads are issued together, so a thread that rebuilds a stream from the
+// counts waits for one round trip per batch rather than one per scan.
+constexpr int kColBatch = 16;
+
 template <typename T>
-__device__ __forceinline__ void write_stream(uint8_t *o, const T *col, int P, const uint4 d, const uint32_t *sl)
+__device__ __forceinline__ void load_column(const T *col, int P, int i0, uint32_t (&x)[kColBatch])
+{
+#pragma unroll
+    for (int u = 0; u < kColBatch; ++u)
+        x[u] = static_cast<uint32_t>(__ldg(col + static_cast<size_t>(i0 + u) * P));
+}
+
+// Write one stream's bytes (header and form payload, spec S2/S3) at o, except
+// the section the encoder staged in the stream's slot (the tANS section of a
+// paired stream, the payload of a sparse stream that was staged whole).  The
+// section's place in the stream (byte offset) and length are returned in
+// sec_at and sec_len (0 when there is none).
+template <typename T>
+__device__ __forceinline__ void write_head(uint8_t *o, const T *col, int P, const uint4 d, uint32_t &sec_at,
+                                           uint32_t &sec_len)
 {
     constexpr uint32_t W = sizeof(T);
     const uint32_t hdr = d.y & 0xFFFFu;     // (bits 16+ of d.y: T for paired, a flag for sparse)
@@ -843,6 +861,8 @@ __device__ __forceinline__ void write_stream(uint8_t *o, const T *col, int P, co
     o[0] = static_cast<uint8_t>(hdr & 0xFFu);
     o[1] = static_cast<uint8_t>(hdr >> 8);
     uint32_t k = 2;
+    sec_at = 0;
+    sec_len = 0;
     auto put = [&](uint32_t v) {
         o[k++] = static_cast<uint8_t>(v & 0xFFu);
         if (W == 2)
@@ -851,43 +871,47 @@ __device__ __forceinline__ void write_stream(uint8_t *o, const T *col, int P, co
     if (form == kConstant) {
         put(d.z & 0xFFFFu);
     } else if (form == kLiteral) {
-        const T *q = col;
-        for (int i = 0; i < kScans; ++i, q += P)
-            put(*q);
-    } else if (form == kSparse && ((d.y >> 16) & 1u)) {
-        const int nbytes = static_cast<int>(d.x) - 2;
-        const uint4 *s4 = reinterpret_cast<const uint4 *>(sl);
-        for (int q = 0; q < nbytes; q += 16) {
-            const uint4 c = __ldcs(s4 + q / 16);
-            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+        for (int i0 = 0; i0 < kScans; i0 += kColBatch) {
+            uint32_t x[kColBatch];
+            load_column(col, P, i0, x);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (q + i < nbytes)
-                    o[k + q + i] = static_cast<uint8_t>(wv[i >> 2] >> (8 * (i & 3)));
+            for (int u = 0; u < kColBatch; ++u)
+                put(x[u]);
         }
+    } else if (form == kSparse && ((d.y >> 16) & 1u)) {
+        sec_at = k;
+        sec_len = d.x - 2u;
     } else if (form == kSparse) {
         const uint32_t nnz = d.z >> 16;
         o[k++] = static_cast<uint8_t>(nnz - 1u);
         uint32_t acc = 0;
         int nacc = 0;
-        const T *q = col;
-        for (int i = 0; i < kScans; ++i, q += P) {
-            if (*q) {
-                acc |= static_cast<uint32_t>(i) << nacc;
-                nacc += 9;
-                while (nacc >= 8) {
-                    o[k++] = static_cast<uint8_t>(acc & 0xFFu);
-                    acc >>= 8;
-                    nacc -= 8;
+        for (int i0 = 0; i0 < kScans; i0 += kColBatch) {
+            uint32_t x[kColBatch];
+            load_column(col, P, i0, x);
+#pragma unroll
+            for (int u = 0; u < kColBatch; ++u) {
+                if (x[u]) {
+                    acc |= static_cast<uint32_t>(i0 + u) << nacc;
+                    nacc += 9;
+                    while (nacc >= 8) {
+                        o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                        acc >>= 8;
+                        nacc -= 8;
+                    }
                 }
             }
         }
         if (nacc > 0)
             o[k++] = static_cast<uint8_t>(acc & 0xFFu);
-        q = col;
-        for (int i = 0; i < kScans; ++i, q += P)
-            if (*q)
-                put(*q);
+        for (int i0 = 0; i0 < kScans; i0 += kColBatch) {
+            uint32_t x[kColBatch];
+            load_column(col, P, i0, x);
+#pragma unroll
+            for (int u = 0; u < kColBatch; ++u)
+                if (x[u])
+                    put(x[u]);
+        }
     } else {
         const int shift = static_cast<int>((hdr >> 8) & 15u);
         const uint32_t base = d.z & 0xFFFFu;
@@ -897,42 +921,46 @@ __device__ __forceinline__ void write_stream(uint8_t *o, const T *col, int P, co
             const uint32_t mask = (1u << shift) - 1u;
             uint32_t acc = 0;
             int nacc = 0;
-            const T *q = col;
-            for (int i = 0; i < kScans; ++i, q += P) {
-                acc |= ((static_cast<uint32_t>(*q) - base) & mask) << nacc;
-                nacc += shift;
-                while (nacc >= 8) {
-                    o[k++] = static_cast<uint8_t>(acc & 0xFFu);
-                    acc >>= 8;
-                    nacc -= 8;
+            for (int i0 = 0; i0 < kScans; i0 += kColBatch) {
+                uint32_t x[kColBatch];
+                load_column(col, P, i0, x);
+#pragma unroll
+                for (int u = 0; u < kColBatch; ++u) {
+                    acc |= ((x[u] - base) & mask) << nacc;
+                    nacc += shift;
+                    while (nacc >= 8) {
+                        o[k++] = static_cast<uint8_t>(acc & 0xFFu);
+                        acc >>= 8;
+                        nacc -= 8;
+                    }
                 }
             }
         }
-        // the tANS section starts at byte 0 of the stream's 16-byte aligned
-        // slot: independent 16-byte loads, then bytes
-        const uint32_t Tbits = d.y >> 16;
-        const int nbytes = static_cast<int>((Tbits + 7u) / 8u);
-        const uint4 *s4 = reinterpret_cast<const uint4 *>(sl);
-        for (int q = 0; q < nbytes; q += 16) {
-            const uint4 c = __ldcs(s4 + q / 16);
-            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (q + i < nbytes)
-                    o[k + q + i] = static_cast<uint8_t>(wv[i >> 2] >> (8 * (i & 3)));
-        }
+        // the tANS section starts at byte 0 of the stream's 16-byte aligned slot
+        sec_at = k;
+        sec_len = ((d.y >> 16) + 7u) / 8u;
     }
 }
 
 constexpr int kCompactThreads = 128;
-constexpr int kCompactBytes = 64 * 1024;   // staged byte range per CTA (dynamic shared memory)
+constexpr int kCompactBytes = 32 * 1024;   // staged byte range per CTA (dynamic shared memory)
+constexpr int kCompactUnroll = 4;          // slot loads a thread has in flight
 
 // a4 (second half): write every stream's bytes at blk_dst[b] + offset.  A CTA
 // takes 128 consecutive pixels of one block, whose streams are contiguous in
-// the payload; when their byte range fits, each thread writes its stream into
-// shared memory (placed congruent to the destination modulo 16) and the CTA
-// stores the range with aligned 16-byte writes, bytes only at the two ragged
-// ends.  Larger ranges (incompressible data) are written in place.
+// the payload.  When their byte range fits, it is assembled in shared memory
+// (placed congruent to the destination modulo 16) and stored with aligned
+// 16-byte writes, bytes only at the two ragged ends:
+//   1. the range is zeroed;
+//   2. each thread writes its stream's own bytes (header, base, raw low bits,
+//      the forms built from the counts);
+//   3. the staged sections of all the CTA's streams are cut into 16-byte
+//      chunks of their slots, numbered across the CTA by a scan, and every
+//      thread takes chunks in turn, kCompactUnroll loads in flight before it
+//      ORs each chunk into place as five shifted words (the bytes around it
+//      belong to other streams or are still zero).
+// A larger range (incompressible data) is written in place, one stream per
+// thread.
 template <typename T>
 __global__ void __launch_bounds__(kCompactThreads) k_enc_compact(const T *__restrict__ counts, int P, int nblk,
                                                                 const uint4 *__restrict__ desc,
@@ -940,6 +968,10 @@ __global__ void __launch_bounds__(kCompactThreads) k_enc_compact(const T *__rest
                                                                 const unsigned long long *__restrict__ blk_dst)
 {
     extern __shared__ __align__(16) uint8_t s_buf[];     // kCompactBytes + 32
+    __shared__ uint32_t s_warp[32];
+    __shared__ uint32_t s_chunk0[kCompactThreads];       // first chunk number of each stream's section
+    __shared__ uint32_t s_at[kCompactThreads];           // section start in s_buf
+    __shared__ uint32_t s_len[kCompactThreads];          // section bytes
     const int b = blockIdx.y;
     const int p0 = blockIdx.x * kCompactThreads;
     const int p1 = min(P, p0 + kCompactThreads);
@@ -950,21 +982,92 @@ __global__ void __launch_bounds__(kCompactThreads) k_enc_compact(const T *__rest
     const uint4 last = desc[static_cast<long long>(b) * P + p1 - 1];
     const uint32_t r0 = first.w, r1 = last.w + last.x;         // the CTA's byte range in the block
     const bool staged = r1 - r0 <= static_cast<uint32_t>(kCompactBytes);
+    const uint4 d = p < p1 ? desc[sid] : make_uint4(0u, 0u, 0u, 0u);
+    const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
+    const uint32_t *sl = slots + static_cast<size_t>(sid) * kSlotWords;
+    if (!staged) {
+        if (d.x) {
+            uint8_t *o = blk + d.w;
+            uint32_t at, len;
+            write_head<T>(o, col, P, d, at, len);
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(sl);
+            for (uint32_t q = 0; q < len; q += 16) {
+                const uint4 c = __ldcs(s4 + q / 16);
+                const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (q + i < len)
+                        o[at + q + i] = static_cast<uint8_t>(wv[i >> 2] >> (8 * (i & 3)));
+            }
+        }
+        return;
+    }
     uint8_t *dst0 = blk + r0;
     const uint32_t mis = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(dst0) & 15u);
-    if (p < p1) {
-        const uint4 d = desc[sid];
-        if (d.x) {
-            const T *col = counts + static_cast<size_t>(b) * kScans * P + p;
-            uint8_t *o = staged ? s_buf + mis + (d.w - r0) : blk + d.w;
-            write_stream<T>(o, col, P, d, slots + static_cast<size_t>(sid) * kSlotWords);
+    const uint32_t span = mis + (r1 - r0);                      // staged bytes from the aligned start
+    for (uint32_t c = threadIdx.x; c * 16 < span; c += kCompactThreads)
+        reinterpret_cast<uint4 *>(s_buf)[c] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    uint32_t at = 0, len = 0;
+    const uint32_t o = mis + (d.w - r0);
+    if (d.x)
+        write_head<T>(s_buf + o, col, P, d, at, len);
+    uint32_t n_chunks;
+    const uint32_t c0 = block_exclusive_scan((len + 15u) / 16u, s_warp, n_chunks);
+    s_chunk0[threadIdx.x] = c0;
+    s_at[threadIdx.x] = o + at;
+    s_len[threadIdx.x] = len;
+    __syncthreads();
+    const uint4 *slot0 = reinterpret_cast<const uint4 *>(slots + static_cast<size_t>(static_cast<long long>(b) * P + p0) *
+                                                                     kSlotWords);
+    for (uint32_t cb = threadIdx.x; cb < n_chunks; cb += kCompactUnroll * kCompactThreads) {
+        uint4 v[kCompactUnroll];
+        int who[kCompactUnroll];
+        uint32_t j[kCompactUnroll];
+#pragma unroll
+        for (int u = 0; u < kCompactUnroll; ++u) {
+            const uint32_t c = cb + u * kCompactThreads;
+            who[u] = -1;
+            if (c < n_chunks) {
+                // the stream whose chunks hold c: the last one starting at or before c
+                int lo = 0, hi = kCompactThreads - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_chunk0[mid] <= c)
+                        lo = mid;
+                    else
+                        hi = mid - 1;
+                }
+                who[u] = lo;
+                j[u] = c - s_chunk0[lo];
+                v[u] = __ldcs(slot0 + static_cast<size_t>(lo) * (kSlotWords / 4) + j[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kCompactUnroll; ++u) {
+            if (who[u] < 0)
+                continue;
+            const uint32_t rem = s_len[who[u]] - 16u * j[u];   // >= 1
+            uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            if (rem < 16u) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int keep = min(4, max(0, static_cast<int>(rem) - 4 * t));
+                    w[t] = keep == 4 ? w[t] : (w[t] & ((1u << (8 * keep)) - 1u));
+                }
+            }
+            const uint32_t a = s_at[who[u]] + 16u * j[u];
+            const uint32_t m = (a & 3u) * 8u;
+            uint32_t *wp = reinterpret_cast<uint32_t *>(s_buf + (a & ~3u));
+#pragma unroll
+            for (int t = 0; t < 5; ++t) {
+                const uint32_t x = __funnelshift_l(t ? w[t - 1] : 0u, t < 4 ? w[t] : 0u, m);
+                if (x)
+                    atomicOr(wp + t, x);
+            }
         }
     }
-    if (!staged)
-        return;
     __syncthreads();
-    const uint32_t len = r1 - r0;
-    const uint32_t span = mis + len;                            // staged bytes from the aligned start
     uint8_t *aligned = dst0 - mis;
     for (uint32_t c = threadIdx.x; c * 16 < span; c += kCompactThreads) {
         const uint32_t lo = c * 16, hi = lo + 16;
@@ -1456,6 +1559,15 @@ __device__ __forceinline__ void index_task(const IndexView &ix, long long b, int
 
 constexpr int kMaxSlots = 8;    // block rows one CTA range may touch (shared accumulators)
 
+// a / b for 0 <= a, 0 < b < 2^32: a 32-bit division when a fits in 32 bits
+// (task numbers of every realistic query), the 64-bit one otherwise
+__device__ __forceinline__ long long qdiv(long long a, long long b)
+{
+    if ((static_cast<unsigned long long>(a) >> 32) == 0ull)
+        return static_cast<long long>(static_cast<uint32_t>(a) / static_cast<uint32_t>(b));
+    return a / b;
+}
+
 template <int W, int THREADS, bool DELTA>
 __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint32_t *__restrict__ dec_g,
                                                              const uint32_t *__restrict__ runs_g,
@@ -1486,6 +1598,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     // launched as a programmatic dependent of the plan: everything above only
     // touched shared memory and the constant tables; wait here until the plan
     // grid has finished and its list, counts and rows are visible
+    for (int i = threadIdx.x; i < kMaxSlots * kScans; i += THREADS)
+        s_acc[i] = 0u;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t n = __ldg(count);          // heavy entries, list[0, n)
     const uint32_t n_l = __ldg(count + 1);    // light entries, list[P - n_l, P)
@@ -1500,9 +1614,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
         constexpr uint32_t K = W == 1 ? 32u : 16u;
         const long long chunks = (n_it + K - 1) / K;
         const long long itotal = rows * chunks;
-        const long long I0 = itotal * blockIdx.x / gridDim.x, I1 = itotal * (blockIdx.x + 1) / gridDim.x;
+        const long long I0 = qdiv(itotal * blockIdx.x, gridDim.x), I1 = qdiv(itotal * (blockIdx.x + 1), gridDim.x);
         for (long long t = I0 + warp0; t < I1; t += MAXW) {
-            const long long row = t / chunks;
+            const long long row = qdiv(t, chunks);
             const int c = static_cast<int>(t - row * chunks);
             index_task<W>(ix, row * stride, c, n_it, row, out, keep, out_bytes, lane0);
         }
@@ -1518,26 +1632,42 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     constexpr long long kMaxCount = W == 1 ? 255 : 65535;
     constexpr long long F = 0x7FFFFFFFll / (32 * kMaxCount);
     const long long nch = (tiles + F - 1) / F;              // pieces per row
-    const long long T0 = total * blockIdx.x / gridDim.x, T1 = total * (blockIdx.x + 1) / gridDim.x;
+    const long long T0 = qdiv(total * blockIdx.x, gridDim.x), T1 = qdiv(total * (blockIdx.x + 1), gridDim.x);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto vrow_of = [&](long long t) {
-        const long long row = t / tiles;
+        const long long row = qdiv(t, tiles);
         return row * nch + (t - row * tiles) / F;
     };
     // tasks of piece vr inside [T0, T1)
     auto piece_tasks = [&](long long vr) {
-        const long long row = vr / nch, c = vr - row * nch;
+        const long long row = qdiv(vr, nch), c = vr - row * nch;
         const long long a = row * tiles + c * F, b = row * tiles + min((c + 1) * F, tiles);
         return max(0ll, min(b, T1) - max(a, T0));
+    };
+    // A share whose pieces all hold a slot from the start may take its tasks
+    // in any order.  It takes the heavy tiles of all its rows first, then the
+    // light ones: a warp that finishes early and takes a second task then
+    // takes a short one, instead of starting a heavy tile late.
+    const long long th = static_cast<long long>((n + 31u) >> 5);
+    const bool heavy_first = T1 > T0 && th > 0 && th < tiles && vrow_of(T1 - 1) - vrow_of(T0) < kMaxSlots;
+    auto task_at = [&](long long k) {       // the k-th task of the share in that order
+        const long long r0 = qdiv(T0, tiles), r1 = qdiv(T1 - 1, tiles);
+        for (int pass = 0; pass < 2; ++pass)
+            for (long long r = r0; r <= r1; ++r) {
+                const long long lo = r == r0 ? T0 - r * tiles : 0, hi = r == r1 ? T1 - r * tiles : tiles;
+                const long long a = pass ? max(lo, th) : lo, b = pass ? hi : min(hi, th);
+                if (k < b - a)
+                    return r * tiles + a + k;
+                k -= max(0ll, b - a);
+            }
+        return T1;
     };
     __shared__ unsigned long long s_next;
     __shared__ long long s_owner[kMaxSlots];
     __shared__ uint32_t s_left[kMaxSlots];
     __shared__ int s_abort;                   // set once a wait ran out: the CTA stops taking tasks
-    for (int i = threadIdx.x; i < kMaxSlots * kScans; i += THREADS)
-        s_acc[i] = 0u;
     if (threadIdx.x == 0) {
-        s_next = static_cast<unsigned long long>(T0);
+        s_next = static_cast<unsigned long long>(T0 + MAXW);
         s_abort = 0;
     }
     if (threadIdx.x < kMaxSlots && T1 > T0) {
@@ -1547,14 +1677,24 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
         s_left[threadIdx.x] = static_cast<uint32_t>(vr <= vrow_of(T1 - 1) ? piece_tasks(vr) : 0);
     }
     __syncthreads();
+    // warp w takes task w of the share first (in heavy-first order the heavy
+    // tiles go to warps 0, 1, 2, ..., spread evenly over the SM's four
+    // schedulers), then the next from the counter
+    bool first_task = true;
     while (true) {
         long long t = 0;
-        if (lane == 0)
-            t = *reinterpret_cast<volatile int *>(&s_abort) ? T1 : static_cast<long long>(atomicAdd(&s_next, 1ull));
+        if (lane == 0) {
+            t = *reinterpret_cast<volatile int *>(&s_abort)
+                    ? T1
+                    : (first_task ? T0 + warp : static_cast<long long>(atomicAdd(&s_next, 1ull)));
+            if (heavy_first && t < T1)
+                t = task_at(t - T0);
+        }
+        first_task = false;
         t = __shfl_sync(kFull, t, 0);
         if (t >= T1)
             break;
-        const long long row = t / tiles;
+        const long long row = qdiv(t, tiles);
         const int tile = static_cast<int>(t - row * tiles);
         const long long vr = row * nch + tile / F;
         const int slot = static_cast<int>(vr & (kMaxSlots - 1));
