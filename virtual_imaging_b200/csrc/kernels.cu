@@ -489,6 +489,19 @@ __global__ void k_generate(T *__restrict__ out, uint64_t seed, int64_t scan0, in
 // ---------------------------------------------------------------------------
 // encoder (a2-a4)
 // ---------------------------------------------------------------------------
+// Counts of scans i0 .. i0 + N - 1 of one pixel column (stride P): the loads
+// are issued together, so a thread that reads a stream's counts waits for one
+// round trip per batch rather than one per scan.
+constexpr int kColBatch = 16;
+
+template <typename T, int N>
+__device__ __forceinline__ void load_column(const T *col, int P, int i0, uint32_t (&x)[N])
+{
+#pragma unroll
+    for (int u = 0; u < N; ++u)
+        x[u] = static_cast<uint32_t>(__ldg(col + static_cast<size_t>(i0 + u) * P));
+}
+
 constexpr int kEncThreads = 256;
 
 // a2+a3: per stream (one thread): statistics, base/shift, hi histogram, model
@@ -497,7 +510,7 @@ constexpr int kEncThreads = 256;
 // and the form decision.  desc: x = length, y = header | T << 16,
 // z = base (or constant value) | nnz << 16, w = offset (filled by layout).
 template <typename T>
-__global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict__ counts, int P, int nblk,
+__global__ void __launch_bounds__(kEncThreads, 6) k_enc_streams(const T *__restrict__ counts, int P, int nblk,
                                                             Tables tb, uint4 *__restrict__ desc,
                                                             uint32_t *__restrict__ slots,
                                                             unsigned long long *__restrict__ stats,
@@ -526,29 +539,38 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
         uint32_t nnz = 0, mn = 0xFFFFFFFFu, mx = 0;
         uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;      // first four nonzeros: scan | value << 16
         // the histogram of the counts below 16 is taken in the same pass: when no
-        // count reaches 16 it is the hi histogram after the base (no shift)
+        // count reaches 16 it is the hi histogram after the base (no shift).  Only
+        // nonzero counts do any work here (most counts of a low-dose pixel are
+        // 0): the zeros' bin, the minimum and the statistics follow from nnz.
 #pragma unroll
-        for (int v = 0; v < 16; ++v)
+        for (int v = 1; v < 16; ++v)
             s_hist[v][tid] = 0;
-        {
-            const T *q = col;
-#pragma unroll 8
-            for (int i = 0; i < kScans; ++i, q += P) {
-                const uint32_t v = *q;
-                if (v < 16u)
-                    s_hist[v][tid] += 1;
-                if (v && nnz < 4u) {
-                    const uint32_t e = static_cast<uint32_t>(i) | (v << 16);
-                    c0 = nnz == 0u ? e : c0;
-                    c1 = nnz == 1u ? e : c1;
-                    c2 = nnz == 2u ? e : c2;
-                    c3 = nnz == 3u ? e : c3;
+        constexpr int kB = 8;           // loads in flight per thread (occupancy bounds the batch)
+        for (int i0 = 0; i0 < kScans; i0 += kB) {
+            uint32_t x[kB];
+            load_column(col, P, i0, x);
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const uint32_t v = x[u];
+                if (v) {
+                    if (v < 16u)
+                        s_hist[v][tid] += 1;
+                    if (nnz < 4u) {
+                        const uint32_t e = static_cast<uint32_t>(i0 + u) | (v << 16);
+                        c0 = nnz == 0u ? e : c0;
+                        c1 = nnz == 1u ? e : c1;
+                        c2 = nnz == 2u ? e : c2;
+                        c3 = nnz == 3u ? e : c3;
+                    }
+                    ++nnz;
+                    mn = min(mn, v);
+                    mx = max(mx, v);
                 }
-                nnz += v != 0u;
-                mn = min(mn, v);
-                mx = max(mx, v);
             }
         }
+        s_hist[0][tid] = static_cast<uint16_t>(kScans - nnz);
+        if (nnz < static_cast<uint32_t>(kScans))
+            mn = 0u;
         uint4 d = make_uint4(0u, 0u, 0u, 0u);
         int form = kEmpty, model = -1;
         if (nnz == 0u) {
@@ -617,26 +639,58 @@ __global__ void __launch_bounds__(kEncThreads) k_enc_streams(const T *__restrict
                     nacc -= 32;
                 }
             };
-            const T *q = col + static_cast<size_t>(kScans - 2) * P;
-            for (int j = kPairs - 1; j >= 0; --j, q -= 2 * static_cast<size_t>(P)) {
-                const bool on_b = two && (j & 1);
-                uint32_t X = on_b ? XB : XA;
-                const uint32_t a = (static_cast<uint32_t>(q[0]) - base) >> shift;
-                const uint32_t bb = (static_cast<uint32_t>(q[P]) - base) >> shift;
+            // one tANS encode step of pair (ca, cb) from state X: the bits to emit
+            // (chunk, k) and the new state
+            auto step = [&](uint32_t ca, uint32_t cb, uint32_t &X, uint32_t &k) {
+                const uint32_t a = (ca - base) >> shift;
+                const uint32_t bb = (cb - base) >> shift;
                 const uint32_t es = __ldg(esym + a + 16u * bb);
                 const uint32_t f = es & 0x7FFu;
                 const uint32_t cum = (es >> 11) & 0x7FFu;
                 const uint32_t k0 = es >> 22;
-                const uint32_t k = k0 - ((X >> k0) < f ? 1u : 0u);
+                k = k0 - ((X >> k0) < f ? 1u : 0u);
                 const uint32_t chunk = X & ((1u << k) - 1u);
                 const uint32_t y = X >> k;
                 X = kStates + __ldg(eslot + cum + (y - f));
-                if (on_b)
-                    XB = X;
-                else
-                    XA = X;
-                push(chunk, k);
-                Tbits += k;
+                return chunk;
+            };
+            // the counts are read again kEB scans at a time, from the top (the
+            // loads of a batch are issued together)
+            constexpr int kEB = 8;
+            if (__all_sync(__activemask(), two)) {
+                // every stream of these lanes has two states: odd pair j on B and
+                // even pair j - 1 on A are independent steps
+                for (int i0 = kScans - kEB; i0 >= 0; i0 -= kEB) {
+                    uint32_t x[kEB];
+                    load_column(col, P, i0, x);
+#pragma unroll
+                    for (int u = kEB / 2 - 1; u > 0; u -= 2) {
+                        uint32_t kb, ka;
+                        const uint32_t cb = step(x[2 * u], x[2 * u + 1], XB, kb);
+                        const uint32_t ca = step(x[2 * u - 2], x[2 * u - 1], XA, ka);
+                        push(cb, kb);
+                        push(ca, ka);
+                        Tbits += kb + ka;
+                    }
+                }
+            } else {
+                for (int i0 = kScans - kEB; i0 >= 0; i0 -= kEB) {
+                    uint32_t x[kEB];
+                    load_column(col, P, i0, x);
+#pragma unroll
+                    for (int u = kEB / 2 - 1; u >= 0; --u) {
+                        const bool on_b = two && (u & 1);     // pair i0 / 2 + u; i0 / 2 is even
+                        uint32_t X = on_b ? XB : XA;
+                        uint32_t k;
+                        const uint32_t chunk = step(x[2 * u], x[2 * u + 1], X, k);
+                        if (on_b)
+                            XB = X;
+                        else
+                            XA = X;
+                        push(chunk, k);
+                        Tbits += k;
+                    }
+                }
             }
             // the section starts with x_A, then x_B: prepended last, in reverse
             if (two)
@@ -831,19 +885,6 @@ __global__ void __launch_bounds__(kLayoutThreads) k_enc_layout(uint4 *__restrict
         if ((lane & 1) == 0)
             rec[1 + lane / 2] = end | (other << 16);
     }
-}
-
-// Counts of scans i0 .. i0 + kColBatch - 1 of one pixel column (stride P):
-// the loads are issued together, so a thread that rebuilds a stream from the
-// counts waits for one round trip per batch rather than one per scan.
-constexpr int kColBatch = 16;
-
-template <typename T>
-__device__ __forceinline__ void load_column(const T *col, int P, int i0, uint32_t (&x)[kColBatch])
-{
-#pragma unroll
-    for (int u = 0; u < kColBatch; ++u)
-        x[u] = static_cast<uint32_t>(__ldg(col + static_cast<size_t>(i0 + u) * P));
 }
 
 // Write one stream's bytes (header and form payload, spec S2/S3) at o, except
