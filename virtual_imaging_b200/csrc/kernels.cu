@@ -1535,18 +1535,15 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
 // most 1024 8-bit counts, or 16 groups of 16-bit counts), so a 64-bit output
 // takes them sign-extended.
 template <int W>
-__device__ __forceinline__ void index_task(const IndexView &ix, long long b, int c, uint32_t n_it, long long row,
+__device__ __forceinline__ void index_task(const IndexView &ix, long long b, uint32_t i0, uint32_t cnt, long long row,
                                            void *out, void *keep, int out_bytes, int lane)
 {
-    constexpr uint32_t K = W == 1 ? 32u : 16u;      // items per task
     uint32_t acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j)
         acc[j] = 0u;
     // lane i fetches item i of the task and its descriptor: one round trip
-    // for all of them
-    const uint32_t i0 = static_cast<uint32_t>(c) * K;
-    const uint32_t cnt = min(K, n_it - i0);
+    // for all of them (cnt <= 32)
     uint32_t my_it = 0u, my_d = 0u;
     if (static_cast<uint32_t>(lane) < cnt) {
         my_it = __ldg(ix.items + i0 + lane);
@@ -1554,15 +1551,13 @@ __device__ __forceinline__ void index_task(const IndexView &ix, long long b, int
         my_d = __ldg(ix.desc + static_cast<long long>(b) * ix.G + g);
     }
     const unsigned long long base = __ldg(ix.base + b);
-    for (uint32_t i = 0; i < cnt; ++i) {
+    // scans lane, lane + 32, ... of item i (zeros for an all-zero group); the
+    // returned mask negates a subtracted item's sums
+    auto fetch = [&](uint32_t i, uint32_t (&v)[16]) {
         const uint32_t d = __shfl_sync(kFull, my_d, static_cast<int>(i));
         const uint32_t it = __shfl_sync(kFull, my_it, static_cast<int>(i));
         const uint32_t code = d >> 30;
-        if (code == 0u)
-            continue;
         const unsigned long long a = base + (d & 0x3FFFFFFFu);
-        const uint32_t sgn = (it >> 31) ? 0xFFFFFFFFu : 0u;     // v -> (v ^ sgn) - sgn negates
-        uint32_t v[16];
         if (code == 1u) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
@@ -1571,14 +1566,32 @@ __device__ __forceinline__ void index_task(const IndexView &ix, long long b, int
 #pragma unroll
             for (int j = 0; j < 16; ++j)
                 v[j] = __ldg(reinterpret_cast<const uint16_t *>(a) + lane + 32 * j);
-        } else {
+        } else if (code == 3u) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
                 v[j] = __ldg(reinterpret_cast<const uint32_t *>(a) + lane + 32 * j);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                v[j] = 0u;
+        }
+        return (it >> 31) ? 0xFFFFFFFFu : 0u;     // v -> (v ^ sgn) - sgn negates
+    };
+    // two items at a time: the loads of both are in flight before either is added
+    for (uint32_t i = 0; i < cnt; i += 2) {
+        uint32_t va[16], vb[16];
+        const uint32_t sa = fetch(i, va);
+        uint32_t sb = 0u;
+        if (i + 1 < cnt) {
+            sb = fetch(i + 1, vb);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                vb[j] = 0u;
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            acc[j] += (v[j] ^ sgn) - sgn;
+            acc[j] += ((va[j] ^ sa) - sa) + ((vb[j] ^ sb) - sb);
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -1647,21 +1660,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
     const long long tiles = ((n + 31u) >> 5) + ((n_l + 31u) >> 5);
     const long long total = rows * tiles;
     const int warp0 = threadIdx.x >> 5, lane0 = threadIdx.x & 31;
-    if (ix.desc != nullptr) {
-        // index items (whole groups inside the mask, or inside its change):
-        // K per task (32, or 16 for 16-bit counts), each lane adding the groups' stored sums of
-        // scans lane, lane + 32, ...; the sums go straight to the output
-        const uint32_t n_it = __ldg(count + 2);
-        constexpr uint32_t K = W == 1 ? 32u : 16u;
-        const long long chunks = (n_it + K - 1) / K;
-        const long long itotal = rows * chunks;
-        const long long I0 = qdiv(itotal * blockIdx.x, gridDim.x), I1 = qdiv(itotal * (blockIdx.x + 1), gridDim.x);
-        for (long long t = I0 + warp0; t < I1; t += MAXW) {
-            const long long row = qdiv(t, chunks);
-            const int c = static_cast<int>(t - row * chunks);
-            index_task<W>(ix, row * stride, c, n_it, row, out, keep, out_bytes, lane0);
-        }
-    }
     // Each CTA owns one contiguous share [T0, T1) of the tasks (row-major:
     // row, then tile); its warps take the next task from a shared counter as
     // they finish, with no barrier between tasks.  Scan sums of a row gather
@@ -1718,6 +1716,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
         s_left[threadIdx.x] = static_cast<uint32_t>(vr <= vrow_of(T1 - 1) ? piece_tasks(vr) : 0);
     }
     __syncthreads();
+    if (ix.desc != nullptr) {
+        // index items (whole groups inside the mask, or inside its change),
+        // before the warp's decode tasks and with no barrier between the two:
+        // K per task, each lane adding the groups' stored sums of scans lane,
+        // lane + 32, ...; the sums go straight to the output.  K is at most 32
+        // (16 for 16-bit counts, so that K root sums stay below 2^31) and is
+        // lowered, down to 4, until the tasks fill the grid's warps: a task's
+        // items are read two at a time, so its time grows with K
+        const uint32_t n_it = __ldg(count + 2);
+        constexpr uint32_t kKMax = W == 1 ? 32u : 16u;
+        const long long want = (static_cast<long long>(n_it) * rows + gridDim.x * MAXW - 1) / (gridDim.x * MAXW);
+        const uint32_t K = static_cast<uint32_t>(max(4ll, min(static_cast<long long>(kKMax), want)));
+        const long long chunks = (n_it + K - 1) / K;
+        const long long itotal = rows * chunks;
+        const long long I0 = qdiv(itotal * blockIdx.x, gridDim.x), I1 = qdiv(itotal * (blockIdx.x + 1), gridDim.x);
+        for (long long t = I0 + warp0; t < I1; t += MAXW) {
+            const long long row = qdiv(t, chunks);
+            const uint32_t i0 = static_cast<uint32_t>(t - row * chunks) * K;
+            index_task<W>(ix, row * stride, i0, min(K, n_it - i0), row, out, keep, out_bytes, lane0);
+        }
+    }
     // warp w takes task w of the share first (in heavy-first order the heavy
     // tiles go to warps 0, 1, 2, ..., spread evenly over the SM's four
     // schedulers), then the next from the counter
