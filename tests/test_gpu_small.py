@@ -306,3 +306,93 @@ def test_uint8_warps_with_base_and_raw_bits():
             img = image(res, drag[t], k, delta=True)
             assert (img == O.dense_masked_sum(x, drag[t], None, k)).all(), (k, t)
     res.free()
+
+
+def _raw_pixel(rng, scans, shift, base):
+    """Counts of one uint8 pixel whose streams carry `shift` raw low bits (spec S3): a
+    lambda = 3 pixel plus `base`, with spikes that set the span of every block."""
+    v = rng.poisson(3.0, size=scans) + base
+    span_lo, span_hi = 1 << (shift + 3), (1 << (shift + 4)) - 1
+    for b0 in range(0, scans, 512):
+        at = rng.choice(np.arange(b0, b0 + 512), size=3, replace=False)
+        v[at] = base + rng.integers(span_lo, min(span_hi, 255 - base) + 1, size=3)
+    return np.minimum(v, 255)
+
+
+def test_uint8_delta_single_raw_lane():
+    """Deltas whose 32-lane tiles hold exactly one stream with raw low bits (the whole
+    warp reads that lane's low bits) or two (each lane reads its own), entering and
+    leaving, with shifts 1-3 and with bases: every image equals the oracle's dense sum."""
+    rng = np.random.default_rng(91)
+    det, scans = 32, 1024
+    P = det * det
+    x = rng.poisson(3.0, size=(scans, P)).astype(np.int64)
+    raw = [40, 77, 131, 250, 301, 402]
+    spec = [(1, 0), (2, 0), (3, 5), (3, 0), (1, 9), (2, 3)]      # (shift, base)
+    for p, (sh, base) in zip(raw, spec):
+        x[:, p] = _raw_pixel(rng, scans, sh, base)
+    x = np.minimum(x, 255).astype(np.uint8)
+    for p, (sh, base) in zip(raw, spec):
+        for b0 in (0, 512):
+            h = O.stream_header(O.encode_stream(x[b0:b0 + 512, p], 1))
+            assert h[0] == 3 and h[2] == sh and h[1] >= 8, (p, h)
+    w = W.Workload("raw1", scans // 32, 32, det, det, 8, 0, "host")
+    res = gpu_encode(w, x)
+    plain = [p for p in range(500, 1024) if p not in raw]
+    m = np.zeros(P, np.uint8)
+    m[plain[:200]] = 1
+    steps = []
+    m1 = m.copy(); m1[[raw[0]] + plain[200:210]] = 1; steps.append(m1)            # one raw lane enters
+    m2 = m1.copy(); m2[[raw[1], raw[2]] + plain[210:215]] = 1; steps.append(m2)   # two raw lanes enter
+    m3 = m2.copy(); m3[[raw[0]] + plain[:3]] = 0; steps.append(m3)                # one raw lane leaves
+    m4 = m3.copy(); m4[raw[1]] = 0; m4[raw[3]] = 1; steps.append(m4)               # one leaves, one enters
+    m5 = m4.copy(); m5[raw[2]] = 0; steps.append(m5)                               # a raw lane alone
+    m6 = m5.copy(); m6[[raw[4], raw[5]]] = 1; m6[plain[100:140]] = 0; steps.append(m6)
+    m7 = m6.copy(); m7[raw[5]] = 0; m7[plain[140:141]] = 0; steps.append(m7)
+    for k in (1, 2):
+        img = image(res, m, k)
+        assert (img == O.dense_masked_sum(x, m, None, k)).all()
+        for t, mt in enumerate(steps):
+            img = image(res, mt, k, delta=True)
+            assert (img == O.dense_masked_sum(x, mt, None, k)).all(), (k, t)
+    res.free()
+
+
+def test_uint8_delta_raw_value_out_of_range():
+    """A raw low bit that lifts a count past 255 (base 225, shift 1, a 255 whose low bit is
+    0, flipped) is malformed for the oracle and for a delta that decodes that stream alone;
+    the same delta on the intact resident is exact."""
+    rng = np.random.default_rng(5)
+    det, scans = 8, 512
+    P = det * det
+    x = rng.poisson(3.0, size=(scans, P)).astype(np.uint8)
+    bad_p, bad_scan = 19, 7
+    v = rng.integers(225, 255, size=scans)
+    v[0], v[bad_scan] = 225, 255
+    x[:, bad_p] = v.astype(np.uint8)
+    enc = O.encode(x, 8)
+    g = enc.groups[0]
+    gi, j = divmod(bad_p, 32)
+    e = lambda t: (int(g[gi, 1 + t // 2]) >> (16 * (t & 1))) & 0xFFFF
+    start = int(g[gi, 0]) + (e(j - 1) if j else 0)
+    end = int(g[gi, 0]) + e(j)
+    h = O.stream_header(bytes(enc.payloads[0][start:start + 2]))
+    assert h[0] == 3 and h[2] == 1 and h[3] == 1 and h[1] >= 8, h
+    bad = enc.payloads[0].copy()
+    bad[start + 3] ^= 0x80                      # raw section after header + base: scan 7, shift 1
+    assert O.decode_stream(bytes(bad[start:end]), 1)[0] != 0
+    assert O.decode_stream(bytes(enc.payloads[0][start:end]), 1)[0] == 0
+    w = W.Workload("rawbad", 1, scans, det, det, 8, 0, "host")
+    m0 = np.zeros(P, np.uint8)
+    m0[:10] = 1
+    m1 = m0.copy()
+    m1[bad_p] = 1
+    for payloads, ok in (([bad], False), (None, True)):
+        res = oracle_resident(w, enc, payloads=payloads)
+        assert (image(res, m0) == O.dense_masked_sum(x, m0)).all()
+        if ok:
+            assert (image(res, m1, delta=True) == O.dense_masked_sum(x, m1)).all()
+        else:
+            with pytest.raises(V.MalformedStream):
+                image(res, m1, delta=True)
+        res.free()

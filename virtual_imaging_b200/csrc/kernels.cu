@@ -1333,10 +1333,34 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     const bool two_lane = S.form == kPaired && !runs && S.two;
     bool fast = plain_warp && two_lane && S.shift == 0 && S.base == 0u;
     bool raw_warp = false;
+    // When exactly one lane of such a warp carries raw low bits, the whole warp
+    // reads them: lane l holds words l, l + 32 and l + 64 of that lane's raw
+    // section (at most 4 bits x 512 scans + the lead), and per 32-scan segment
+    // each lane extracts the low bits of its own scan.  The raw lane's table
+    // steps are shifted like every other lane's; its low bits join the scan
+    // sums after the warp reduction.  (The raw lane alone would spend ~16
+    // instructions per pair on them, the whole warp waiting.)
+    int coop_r = -1;
+    uint32_t rw0 = 0u, rw1 = 0u, rw2 = 0u, r_lead = 0u, r_shift = 0u;
+    bool r_neg = false;
     if constexpr (W == 1 && ROOMY) {
         const bool all_two = __all_sync(kFull, !(S.form == kPaired && !runs) || S.two);
         raw_warp = __any_sync(kFull, two_lane && (S.shift != 0 || S.base != 0u));
         fast = all_two && two_lane;
+        const unsigned rm = __ballot_sync(kFull, all_two && two_lane && S.shift != 0);
+        if (__popc(rm) == 1) {
+            coop_r = __ffs(rm) - 1;
+            const unsigned long long f =
+                __shfl_sync(kFull, reinterpret_cast<unsigned long long>(S.br.first), coop_r);
+            const uint32_t li = __shfl_sync(kFull, S.br.li, coop_r);
+            r_lead = __shfl_sync(kFull, static_cast<uint32_t>(S.br.lead), coop_r);
+            r_shift = __shfl_sync(kFull, static_cast<uint32_t>(S.shift), coop_r);
+            r_neg = __shfl_sync(kFull, neg ? 1u : 0u, coop_r) != 0u;
+            const uint32_t *fw = reinterpret_cast<const uint32_t *>(f);
+            rw0 = __ldg(fw + min(static_cast<uint32_t>(lane), li));
+            rw1 = __ldg(fw + min(static_cast<uint32_t>(lane) + 32u, li));
+            rw2 = __ldg(fw + min(static_cast<uint32_t>(lane) + 64u, li));
+        }
     }
     uint32_t over = 0;
     // warps whose lanes hold only empty, sparse or run-decoded streams skip the per-scan loop
@@ -1373,7 +1397,17 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                     pk[jj + 1] = consume(eb, S.x2, S.bt.lo, S.bt.hi, S.bt.n);
                 }
                 if constexpr (W == 1 && ROOMY) {
-                  if (raw_warp) {
+                  if (raw_warp && coop_r >= 0) {
+                    // v = base + (hi << shift), both halves at once; the raw lane's
+                    // low bits are added after the reduction (below)
+                    const uint32_t bpk = S.base | (S.base << 16);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const uint32_t v = (pk[jj] << S.shift) + bpk;
+                        over |= (v & 0xFFFFu) | (v >> 16);
+                        pk[jj] = v;
+                    }
+                  } else if (raw_warp) {
                     // v = base + (hi << shift | lo), both halves at once
                     const uint32_t m = (1u << S.shift) - 1u;
                     const uint32_t bpk = S.base | (S.base << 16);
@@ -1408,6 +1442,38 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                 for (int jj = 0; jj < 16; ++jj)
                     pk[jj] = cpk;
             }
+            uint32_t lo_add = 0u;
+            if constexpr (W == 1 && ROOMY) {
+                if (coop_r >= 0) {
+                    // (warp-uniform: every lane takes part, whatever its own stream)
+                    // the raw lane's value of scan seg * 32 + lane without its low
+                    // bits, through shared memory; then the low bits of that scan
+                    // from the words the lanes hold, and the full value's range check
+                    if (lane == coop_r) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            stage[jj] = pk[jj];
+                    }
+                    __syncwarp();
+                    const uint32_t vw = stage[lane >> 1];
+                    __syncwarp();
+                    const uint32_t vp = (lane & 1) ? (vw >> 16) : (vw & 0xFFFFu);
+                    const uint32_t bit = r_lead + static_cast<uint32_t>(seg * 32 + lane) * r_shift;
+                    const uint32_t k0 = bit >> 5, k1 = k0 + 1u;
+                    const uint32_t a0 = __shfl_sync(kFull, rw0, static_cast<int>(k0 & 31u));
+                    const uint32_t a1 = __shfl_sync(kFull, rw1, static_cast<int>(k0 & 31u));
+                    const uint32_t a2 = __shfl_sync(kFull, rw2, static_cast<int>(k0 & 31u));
+                    const uint32_t b0 = __shfl_sync(kFull, rw0, static_cast<int>(k1 & 31u));
+                    const uint32_t b1 = __shfl_sync(kFull, rw1, static_cast<int>(k1 & 31u));
+                    const uint32_t b2 = __shfl_sync(kFull, rw2, static_cast<int>(k1 & 31u));
+                    const uint32_t w0 = k0 < 32u ? a0 : (k0 < 64u ? a1 : a2);
+                    const uint32_t w1 = k1 < 32u ? b0 : (k1 < 64u ? b1 : b2);
+                    const uint32_t lo = __funnelshift_r(w0, w1, bit & 31u) & ((1u << r_shift) - 1u);
+                    if (vp + lo > 0xFFu)
+                        report(st, kErrValue);
+                    lo_add = r_neg ? 0u - lo : lo;
+                }
+            }
             // warp sums of the 16 packed pairs are warp-uniform: one lane
             // parks them in shared memory, every lane then takes its scan
 #pragma unroll
@@ -1419,7 +1485,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
             __syncwarp();
             uint32_t mine = stage[lane >> 1];
             __syncwarp();
-            mine = ((lane & 1) ? (mine >> 16) : (mine & 0xFFFFu)) - (DELTA ? corr : 0u);
+            mine = ((lane & 1) ? (mine >> 16) : (mine & 0xFFFFu)) - (DELTA ? corr : 0u) + lo_add;
             if (mine)
                 atomicAdd(acc + seg * 32 + lane, mine);
         }
