@@ -496,6 +496,9 @@ def run_profile_case(dev, torch, V):
     frames = torch.empty((2 * 512, w.n_pixels), dtype=torch.uint8, device=dev)
     res.decode_blocks(0, 2, out=frames)
     res.decode_range(777, 1)
+    # launch 14: bright field with the index dropped (every disk pixel decoded pair by pair)
+    res.drop_index()
+    res.masked_sum(bf, out=out)
     p = res.profile_read()
     print(json.dumps({"encode_s": t_enc, "kernels": p}), flush=True)
     res.free()
