@@ -470,15 +470,16 @@ def run_profile_encode(dev, torch, V):
     res.free()
 
 
-def run_profile_case(dev, torch, V):
-    """Small bounded case for ncu: build the default resident, then a few bright-field / annular
-    block_stride-1 queries (the kernels ncu captures are the k_decode_reduce launches)."""
-    w = W.workload("c4")
+def run_profile_case(dev, torch, V, config="c4"):
+    """Small bounded case for ncu: build the resident of `config` (the default workload unless
+    --config names another), then a few bright-field / annular block_stride-1 queries (the
+    kernels ncu captures are the k_decode_reduce launches)."""
+    w = W.workload(config)
     res, buf, t_enc = build_resident(w, dev, torch, V)
     del buf
     torch.cuda.empty_cache()
     res.build_index((w.det_rows // 2, w.det_cols // 2))
-    out = torch.empty((w.n_blocks, 512), dtype=V.out_dtype(32), device=dev)
+    out = torch.empty((w.n_blocks, 512), dtype=V.out_dtype(res.info()["out_bits_auto"]), device=dev)
     bf = torch.from_numpy(w.masks["bf"]).to(dev)
     adf = torch.from_numpy(w.masks["adf"]).to(dev)
     res.profile(True)
@@ -493,7 +494,7 @@ def run_profile_case(dev, torch, V):
         for m in (bf, adf):
             res.masked_sum(m, block_stride=k, out=out[: -(-w.n_blocks // k)])
     # a two-block decode and one frame (k_decode_blocks, k_decode_range)
-    frames = torch.empty((2 * 512, w.n_pixels), dtype=torch.uint8, device=dev)
+    frames = torch.empty((2 * 512, w.n_pixels), dtype=torch.uint8 if w.dtype_bits == 8 else torch.uint16, device=dev)
     res.decode_blocks(0, 2, out=frames)
     res.decode_range(777, 1)
     # launch 14: bright field with the index dropped (every disk pixel decoded pair by pair)
@@ -540,7 +541,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     if args.profile:
-        run_profile_case(dev, torch, V)
+        run_profile_case(dev, torch, V, args.config)
         return
     if args.profile_encode:
         run_profile_encode(dev, torch, V)

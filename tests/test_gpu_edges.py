@@ -111,6 +111,16 @@ def test_zero_block_decode_and_argument_errors(c2):
         res.masked_sum(m, out_bits=64, out=bad.view(w.n_blocks, 512))
     with pytest.raises(V.QemError):                  # 16 is not a width
         res.masked_sum(m, out_bits=16)
+    # an output buffer narrower or shorter than ceil(B/k) x 512 values of the chosen
+    # width is refused before the library could write past it
+    narrow = torch.empty((w.n_blocks, 512), dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        res.masked_sum(m, out_bits=64, out=narrow)
+    short = torch.empty((w.n_blocks - 1, 512), dtype=V.out_dtype(res.info()["out_bits_auto"]), device="cuda")
+    with pytest.raises(ValueError):
+        res.masked_sum_delta(m, out=short)
+    with pytest.raises(ValueError):
+        res.masked_sum_noalloc(m, short)
     res.free()
     part = V.Resident.create((w.scan_rows, w.scan_cols), (w.det_rows, w.det_cols), 16)
     part.append(to_dev(x[:512]), 1)

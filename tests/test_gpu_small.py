@@ -396,3 +396,49 @@ def test_uint8_delta_raw_value_out_of_range():
             with pytest.raises(V.MalformedStream):
                 image(res, m1, delta=True)
         res.free()
+
+
+def test_uint16_raw_value_out_of_range():
+    """uint16: a raw low bit that lifts a count past 65535 (base 65505, shift 1, a 65535 whose
+    low bit is 0, flipped) is malformed for the oracle, for a full query and for a delta
+    that decode that stream; on the intact resident both are exact.  The pixel's other
+    counts are high, so its warp's segments are reduced scan by scan."""
+    rng = np.random.default_rng(6)
+    det, scans = 8, 512
+    P = det * det
+    x = rng.poisson(3.0, size=(scans, P)).astype(np.uint16)
+    bad_p, bad_scan = 37, 9
+    v = rng.integers(65505, 65535, size=scans)
+    v[0], v[bad_scan] = 65505, 65535
+    x[:, bad_p] = v.astype(np.uint16)
+    enc = O.encode(x, 16)
+    g = enc.groups[0]
+    gi, j = divmod(bad_p, 32)
+    e = lambda t: (int(g[gi, 1 + t // 2]) >> (16 * (t & 1))) & 0xFFFF
+    start = int(g[gi, 0]) + (e(j - 1) if j else 0)
+    end = int(g[gi, 0]) + e(j)
+    h = O.stream_header(bytes(enc.payloads[0][start:start + 2]))
+    assert h[0] == 3 and h[2] == 1 and h[3] == 1 and h[1] >= 8, h
+    bad = enc.payloads[0].copy()
+    bad[start + 4 + 1] ^= 0x02                  # raw section after header + 2-byte base: scan 9 = byte 1, bit 1
+    assert O.decode_stream(bytes(bad[start:end]), 2)[0] != 0
+    assert O.decode_stream(bytes(enc.payloads[0][start:end]), 2)[0] == 0
+    w = W.Workload("rawbad16", 1, scans, det, det, 16, 0, "host")
+    m0 = np.zeros(P, np.uint8)
+    m0[:10] = 1
+    m1 = m0.copy()
+    m1[bad_p] = 1
+    for payloads, ok in (([bad], False), (None, True)):
+        res = oracle_resident(w, enc, payloads=payloads)
+        assert (image(res, m0) == O.dense_masked_sum(x, m0)).all()
+        if ok:
+            assert (image(res, m1, delta=True) == O.dense_masked_sum(x, m1)).all()
+            assert (image(res, m1) == O.dense_masked_sum(x, m1)).all()
+        else:
+            with pytest.raises(V.MalformedStream):
+                image(res, m1, delta=True)
+        res.free()
+    res = oracle_resident(w, enc, payloads=[bad])
+    with pytest.raises(V.MalformedStream):
+        image(res, m1)
+    res.free()

@@ -236,6 +236,15 @@ class Resident:
             rows = -(-n_blocks // block_stride)
             bits = auto if out_bits == 0 else out_bits
             out = torch.empty((rows, 512), dtype=out_dtype(bits), device=mask.device)
+        elif block_stride >= 1 and out_bits in (0, 32, 64):
+            # the library writes ceil(B/k) x 512 values of the chosen width through a raw
+            # pointer: a smaller or narrower buffer is refused here (other arguments are
+            # the library's to refuse)
+            n_blocks, _, _, auto = self._static()
+            rows = -(-n_blocks // block_stride)
+            bits = auto if out_bits == 0 else out_bits
+            if out.dtype != out_dtype(bits) or out.numel() < rows * 512:
+                raise ValueError(f"{name}: out must hold {rows} x 512 {out_dtype(bits)} values")
         _check(fn(self._h, _dev_ptr(mask), block_stride, out_bits, _dev_ptr(out), None,
                   1 if wait else 0, _stream(stream)), name)
         return out
@@ -263,6 +272,11 @@ class Resident:
         """Masked sum that allocates no device memory (qem_masked_sum_noalloc): for callers that
         must not allocate while querying.  `out` must be preallocated ([ceil(B/k)][512] of the
         chosen width); calls that overlap on the GPU race on the library's fixed working memory."""
+        if block_stride >= 1 and out_bits in (0, 32, 64):
+            n_blocks, _, _, auto = self._static()
+            bits = auto if out_bits == 0 else out_bits
+            if out.dtype != out_dtype(bits) or out.numel() < -(-n_blocks // block_stride) * 512:
+                raise ValueError("qem_masked_sum_noalloc: out must hold ceil(B/k) x 512 values of the chosen width")
         _check(lib().qem_masked_sum_noalloc(self._h, _dev_ptr(mask), block_stride, out_bits, _dev_ptr(out),
                                             _stream(stream)), "qem_masked_sum_noalloc")
         return out

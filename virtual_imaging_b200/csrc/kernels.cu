@@ -1372,12 +1372,12 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     int coop_r = -1;
     uint32_t rw0 = 0u, rw1 = 0u, rw2 = 0u, r_lead = 0u, r_shift = 0u;
     bool r_neg = false;
-    if constexpr (W == 1 && ROOMY) {
+    if constexpr (ROOMY) {
         const bool all_two = __all_sync(kFull, !(S.form == kPaired && !runs) || S.two);
         raw_warp = __any_sync(kFull, two_lane && (S.shift != 0 || S.base != 0u));
         fast = all_two && two_lane;
         const unsigned rm = __ballot_sync(kFull, all_two && two_lane && S.shift != 0);
-        if (__popc(rm) == 1) {
+        if (W == 1 && __popc(rm) == 1) {
             coop_r = __ffs(rm) - 1;
             const unsigned long long f =
                 __shfl_sync(kFull, reinterpret_cast<unsigned long long>(S.br.first), coop_r);
@@ -1395,17 +1395,20 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     // warps whose lanes hold only empty, sparse or run-decoded streams skip the per-scan loop
     const bool dense = __any_sync(kFull, dense_lane);
 
-    // A uint16 warp whose dense lanes all carry values of at most 255 (paired
-    // streams without base or raw bits, whose values are table symbols, and
-    // small constants) takes the packed uint8 path as well.
+    // A uint16 warp whose dense lanes are all two-state paired streams (with or,
+    // in the kernels with room for it, without a base and raw low bits) or small
+    // constants takes the packed path as well: a segment whose values all stay
+    // below kPackMax + 1 is reduced in packed halves, any other segment scan by
+    // scan (32 lanes x kPackMax must fit a 16-bit half).
+    constexpr uint32_t kPackMax = W == 1 ? 255u : 2047u;
     const bool packed = W == 1 || __all_sync(kFull, !dense_lane || fast || (S.form == kConstant && S.c <= 255u));
     if (packed) {
         // counts fit 16-bit halves: pack scans (2j, 2j+1) into one word; a
-        // leaving pixel contributes 255 - v per half and the warp subtracts
-        // 255 x (number of such lanes) afterwards.
+        // leaving pixel contributes kPackMax - v per half and the warp subtracts
+        // kPackMax x (number of such lanes) afterwards.
         const bool packed_src = dense_lane;
-        const uint32_t flip = (neg && packed_src) ? 0x00FF00FFu : 0u;
-        const uint32_t corr = 255u * static_cast<uint32_t>(__popc(__ballot_sync(kFull, neg && packed_src)));
+        const uint32_t flip = (neg && packed_src) ? (kPackMax | (kPackMax << 16)) : 0u;
+        const uint32_t corr = kPackMax * static_cast<uint32_t>(__popc(__ballot_sync(kFull, neg && packed_src)));
         const uint32_t cpk = S.form == kConstant ? (S.c | (S.c << 16)) : 0u;
         const uint32_t dec_sa = static_cast<uint32_t>(__cvta_generic_to_shared(dec));
         for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
@@ -1425,8 +1428,8 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                         S.bt.refill();
                     pk[jj + 1] = consume(eb, S.x2, S.bt.lo, S.bt.hi, S.bt.n);
                 }
-                if constexpr (W == 1 && ROOMY) {
-                  if (raw_warp && coop_r >= 0) {
+                if constexpr (ROOMY) {
+                  if (W == 1 && raw_warp && coop_r >= 0) {
                     // v = base + (hi << shift), both halves at once; the raw lane's
                     // low bits are added after the reduction (below)
                     const uint32_t bpk = S.base | (S.base << 16);
@@ -1436,7 +1439,7 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                         over |= (v & 0xFFFFu) | (v >> 16);
                         pk[jj] = v;
                     }
-                  } else if (raw_warp) {
+                  } else if (raw_warp && W == 1) {
                     // v = base + (hi << shift | lo), both halves at once
                     const uint32_t m = (1u << S.shift) - 1u;
                     const uint32_t bpk = S.base | (S.base << 16);
@@ -1448,6 +1451,20 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                         const uint32_t v = ((pk[jj] << S.shift) | (lo & m) | (((lo >> S.shift) & m) << 16)) + bpk;
                         over |= (v & 0xFFFFu) | (v >> 16);
                         pk[jj] = v;
+                    }
+                  } else if (raw_warp) {
+                    // uint16: each half on its own (a malformed stream's value
+                    // past 65535 must not carry into the other half unseen)
+                    const uint32_t m = (1u << S.shift) - 1u;
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        if (S.br.n < 2 * S.shift)
+                            S.br.refill();
+                        const uint32_t lo = S.br.get(2 * S.shift);
+                        const uint32_t va = (((pk[jj] & 0xFFFFu) << S.shift) | (lo & m)) + S.base;
+                        const uint32_t vb = (((pk[jj] >> 16) << S.shift) | ((lo >> S.shift) & m)) + S.base;
+                        over |= va | vb;
+                        pk[jj] = va | (vb << 16);
                     }
                   }
                 }
@@ -1501,6 +1518,26 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
                     if (vp + lo > 0xFFu)
                         report(st, kErrValue);
                     lo_add = r_neg ? 0u - lo : lo;
+                }
+            }
+            if constexpr (W == 2 && ROOMY) {
+                // a segment with a value above kPackMax is reduced scan by scan
+                uint32_t so = 0u;
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj)
+                    so |= pk[jj];
+                if (__any_sync(kFull, ((so | (so >> 16)) & 0xFFFFu) > kPackMax)) {
+                    uint32_t mine = 0u;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t v = (i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xFFFFu);
+                        const uint32_t r = __reduce_add_sync(kFull, neg ? 0u - v : v);
+                        if (lane == i)
+                            mine = r;
+                    }
+                    if (mine)
+                        acc_add<ACC_SHARED>(acc + seg * 32 + lane, mine);
+                    continue;
                 }
             }
             // warp sums of the 16 packed pairs are warp-uniform: one lane
@@ -1878,7 +1915,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_decode_reduce(View v, const uint
         // no other piece's sums are flushed into this row
         if (!ok)
             continue;
-        decode_task<W, DELTA, (THREADS <= 512 && DELTA), true>(v, s_dec, dec_g, skip_models, list, n, n_l, tile,
+        decode_task<W, DELTA, (THREADS <= 512 && (DELTA || W == 2)), true>(v, s_dec, dec_g, skip_models, list, n, n_l, tile,
                                                                row * stride, s_acc + slot * kScans, s_stage + warp * 16,
                                                                s_cnt, &s_bar, ready, lane, st);
         // this warp's slot additions happen before its count
