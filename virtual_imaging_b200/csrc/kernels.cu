@@ -1354,15 +1354,16 @@ __device__ __forceinline__ void decode_task(const View &v, const uint32_t *s_dec
     // the general step on all its paired lanes: with both kinds in one warp
     // the fast loop and the general loop would run one after the other.
     const bool plain_warp = __all_sync(kFull, !(S.form == kPaired && !runs) || (S.shift == 0 && S.base == 0u));
-    // uint8: a warp whose pair-by-pair lanes all use two-state models takes the
-    // two-state loop even when some lanes carry a base or raw low bits (one
-    // count of 16 or more in a low-count stream is enough): those are added
-    // per pair after the table steps (8-bit values keep the packed halves apart)
-    // (kernels launched with room for more registers per thread only)
+    // In the kernels launched with room for more registers per thread (uint8
+    // deltas, every uint16 query), a warp whose pair-by-pair lanes all use
+    // two-state models takes the two-state loop even when some lanes carry a
+    // base or raw low bits (one count of 16 or more in a low-count stream is
+    // enough; every high-dose uint16 pixel): those are added per pair after the
+    // table steps, each half on its own for uint16 (a value is at most 65535).
     const bool two_lane = S.form == kPaired && !runs && S.two;
     bool fast = plain_warp && two_lane && S.shift == 0 && S.base == 0u;
     bool raw_warp = false;
-    // When exactly one lane of such a warp carries raw low bits, the whole warp
+    // uint8: when exactly one lane of such a warp carries raw low bits, the whole warp
     // reads them: lane l holds words l, l + 32 and l + 64 of that lane's raw
     // section (at most 4 bits x 512 scans + the lead), and per 32-scan segment
     // each lane extracts the low bits of its own scan.  The raw lane's table
