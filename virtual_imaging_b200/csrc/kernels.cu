@@ -2188,16 +2188,22 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
 // stream's 512 counts in order and stores them down its pixel column of the
 // [n * 512][P] frames (neighbouring threads hold neighbouring pixels, so each
 // scan's stores are coalesced).  Invalid pixels come out 0.
+constexpr int kBlockDecodeThreads = 768;   // 80 registers per thread: the decode loops without spills
+
 template <int W>
-__global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_t *__restrict__ dec_g,
-                                                          long long first, long long nblk, void *__restrict__ out,
-                                                          DevStatus *__restrict__ st)
+__global__ void __launch_bounds__(kBlockDecodeThreads, 1) k_decode_blocks(View v, const uint32_t *__restrict__ dec_g,
+                                                          const uint32_t *__restrict__ runs_g, uint32_t skip_models,
+                                                          int skip_count, long long first, long long nblk,
+                                                          void *__restrict__ out, DevStatus *__restrict__ st)
 {
     using T = typename std::conditional<W == 1, uint8_t, uint16_t>::type;
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *s_dec = smem;
+    // the run-event tables of the low-dose models, then the other decode tables
     for (int i = threadIdx.x; i < kModels * kStates / 4; i += blockDim.x)
-        reinterpret_cast<uint4 *>(s_dec)[i] = __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
+        reinterpret_cast<uint4 *>(s_dec)[i] = i < skip_count * kStates / 4
+                                                  ? __ldg(reinterpret_cast<const uint4 *>(runs_g) + i)
+                                                  : __ldg(reinterpret_cast<const uint4 *>(dec_g) + i);
     __syncthreads();
     T *o = reinterpret_cast<T *>(out);
     const long long total = nblk * v.P;
@@ -2225,8 +2231,66 @@ __global__ void __launch_bounds__(1024, 1) k_decode_blocks(View v, const uint32_
             ok = open_stream(S, W, st);
         if (!ok)
             S.form = kEmpty;
-        if (S.form == kPaired) {
-            const uint32_t *dec = s_dec + S.model * kStates;
+        const bool run_model = (skip_models >> S.model) & 1u;
+        if (S.form == kPaired && run_model && S.shift == 0 && S.base == 0u) {
+            // a low-dose stream: zeros down the column, then its run events (as
+            // in the masked sum: jump the zero-bit (0,0) steps, take the step at
+            // the slot reached) store its nonzero counts
+            for (int i = 0; i < kScans; ++i)
+                dst[i * P] = 0;
+            const uint32_t rt_sa = static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + S.model * kStates));
+            int j = 0;
+            bool bad = false;
+            while (j < kPairs) {
+                const uint32_t t = tab_load(S.x, rt_sa);
+                j += static_cast<int>((t >> 14) & 63u);
+                if (j >= kPairs) {
+                    bad = j > kPairs;
+                    S.x = (t >> 28) & 1u;
+                    break;
+                }
+                if (S.bt.n < 10)
+                    S.bt.refill();
+                S.x = (t & 1023u) | S.bt.get(static_cast<int>((t >> 10) & 15u));
+                const uint32_t a = (t >> 20) & 15u, c = (t >> 24) & 15u;
+                if (a)
+                    dst[static_cast<size_t>(2 * j) * P] = static_cast<T>(a);
+                if (c)
+                    dst[static_cast<size_t>(2 * j + 1) * P] = static_cast<T>(c);
+                ++j;
+            }
+            if (bad)
+                report(st, kErrState);
+            else
+                close_paired(S, st);
+        } else if (S.form == kPaired && S.two && S.shift == 0 && S.base == 0u) {
+            // a two-state stream without base or raw bits (models 8-31, whose
+            // decode tables are in shared memory): both states' table steps
+            // interleaved as in the masked sum, the counts stored as they come
+            const uint32_t dec_sa = static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + S.model * kStates));
+            for (int seg = 0; seg < 16; ++seg) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; jj += 2) {
+                    const uint32_t ea = tab_load(S.x, dec_sa);
+                    const uint32_t eb = tab_load(S.x2, dec_sa);
+                    if (jj % 3 == 0 && S.bt.n < 30)
+                        S.bt.refill();
+                    pk[jj] = consume(ea, S.x, S.bt.lo, S.bt.hi, S.bt.n);
+                    if ((jj + 1) % 3 == 0 && S.bt.n < 30)
+                        S.bt.refill();
+                    pk[jj + 1] = consume(eb, S.x2, S.bt.lo, S.bt.hi, S.bt.n);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    dst[static_cast<size_t>(seg * 32 + 2 * jj) * P] = static_cast<T>(pk[jj] & 0xFFFFu);
+                    dst[static_cast<size_t>(seg * 32 + 2 * jj + 1) * P] = static_cast<T>(pk[jj] >> 16);
+                }
+            }
+            close_paired(S, st);
+        } else if (S.form == kPaired) {
+            // the run-decoded models' decode tables stay in global memory
+            const uint32_t *dec = (run_model ? dec_g : s_dec) + S.model * kStates;
             uint32_t over = 0;
             for (int seg = 0; seg < 16; ++seg) {
                 uint32_t vv[32];
@@ -2886,10 +2950,13 @@ cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n
                                    : ensure_smem(reinterpret_cast<const void *>(k_decode_blocks<2>), smem);
     if (e != cudaSuccess)
         return e;
+    const int skip_count = __builtin_popcount(tb.skip_models);
     if (v.w == 1)
-        k_decode_blocks<1><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
+        k_decode_blocks<1><<<grid, kBlockDecodeThreads, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                                                                    first, n, out, status);
     else
-        k_decode_blocks<2><<<grid, 1024, smem, st>>>(v, tb.dec, first, n, out, status);
+        k_decode_blocks<2><<<grid, kBlockDecodeThreads, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                                                                    first, n, out, status);
     return cudaGetLastError();
 }
 
