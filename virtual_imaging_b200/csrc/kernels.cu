@@ -2053,10 +2053,32 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
             const bool dense_lane = (S.form == kPaired && !runs) || S.form == kLiteral || S.form == kConstant;
             const bool dense = __any_sync(kFull, dense_lane);
             const uint32_t *dec = (run_model ? dec_g : s_dec) + S.model * kStates;
+            // a warp whose pair-by-pair lanes are all two-state streams without
+            // base or raw bits runs their interleaved table steps (models 8-31,
+            // tables in shared memory) instead of the general step
+            const bool two_plain = S.form == kPaired && !runs && S.two && S.shift == 0 && S.base == 0u;
+            const bool fast_warp = __all_sync(kFull, !(S.form == kPaired && !runs) || two_plain);
+            const uint32_t dec_sa = static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + S.model * kStates));
             uint32_t over = 0;
             for (int seg = 0; seg < (dense ? 16 : 0); ++seg) {
                 uint32_t vv[32];
-                if (S.form == kPaired && !runs) {
+                if (fast_warp && two_plain) {
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj += 2) {
+                        const uint32_t ea = tab_load(S.x, dec_sa);
+                        const uint32_t eb = tab_load(S.x2, dec_sa);
+                        if (jj % 3 == 0 && S.bt.n < 30)
+                            S.bt.refill();
+                        const uint32_t pa = consume(ea, S.x, S.bt.lo, S.bt.hi, S.bt.n);
+                        if ((jj + 1) % 3 == 0 && S.bt.n < 30)
+                            S.bt.refill();
+                        const uint32_t pb = consume(eb, S.x2, S.bt.lo, S.bt.hi, S.bt.n);
+                        vv[2 * jj] = pa & 0xFFFFu;
+                        vv[2 * jj + 1] = pa >> 16;
+                        vv[2 * jj + 2] = pb & 0xFFFFu;
+                        vv[2 * jj + 3] = pb >> 16;
+                    }
+                } else if (S.form == kPaired && !runs) {
                     paired_segment(S, dec, vv, over);
                 } else if (S.form == kLiteral) {
 #pragma unroll
@@ -2104,11 +2126,13 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
             if (runs) {
                 // one event per iteration (see decode_task): jump the zero-bit run,
                 // then the landing slot's step; its nonzero counts scatter
-                const uint32_t *rt = s_dec + S.model * kStates;
+                // (the next event's entry is read before this event's additions,
+                // as in the masked sum)
+                const uint32_t rt_sa = static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + S.model * kStates));
                 int j = 0;
                 bool bad = false;
+                uint32_t t = tab_load_ordered(S.x, rt_sa);
                 while (j < kPairs) {
-                    const uint32_t t = rt[S.x];
                     j += static_cast<int>((t >> 14) & 63u);
                     if (j >= kPairs) {
                         bad = j > kPairs;
@@ -2118,6 +2142,7 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
                     if (S.bt.n < 10)
                         S.bt.refill();
                     S.x = (t & 1023u) | S.bt.get(static_cast<int>((t >> 10) & 15u));
+                    const uint32_t tn = tab_load_ordered(S.x, rt_sa);
                     const long long a = (t >> 20) & 15u, c = (t >> 24) & 15u;
                     if (a) {
                         atomicAdd(s_acc + 2 * j, static_cast<unsigned long long>(a * wr));
@@ -2130,6 +2155,7 @@ __global__ void __launch_bounds__(512, 1) k_moments(View v, const uint32_t *__re
                         atomicAdd(s_acc + 2 * kScans + 2 * j + 1, static_cast<unsigned long long>(c));
                     }
                     ++j;
+                    t = tn;
                 }
                 if (bad)
                     report(st, kErrState);
