@@ -2388,15 +2388,16 @@ __global__ void __launch_bounds__(kBlockDecodeThreads, 1) k_decode_blocks(View v
 // stream's extent).  Invalid pixels come out 0.
 template <int W>
 __global__ void __launch_bounds__(256) k_decode_range(View v, const uint32_t *__restrict__ dec_g,
-                                                     long long first, long long n, void *__restrict__ out,
-                                                     DevStatus *__restrict__ st)
+                                                     const uint32_t *__restrict__ runs_g, uint32_t skip_models,
+                                                     int skip_count, long long first, long long n,
+                                                     void *__restrict__ out, DevStatus *__restrict__ st)
 {
     using T = typename std::conditional<W == 1, uint8_t, uint16_t>::type;
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t *s_dec = smem;
     __shared__ __align__(8) uint64_t s_bar;
     if (threadIdx.x == 0)
-        tables_start(&s_bar, s_dec, dec_g, dec_g, 0);
+        tables_start(&s_bar, s_dec, dec_g, runs_g, skip_count);
     __syncthreads();
     bool ready = false;
     T *o = reinterpret_cast<T *>(out);
@@ -2436,8 +2437,63 @@ __global__ void __launch_bounds__(256) k_decode_range(View v, const uint32_t *__
                 ready = true;
             }
         }
-        if (S.form == kPaired) {
-            const uint32_t *dec = s_dec + S.model * kStates;
+        const bool run_model = (skip_models >> S.model) & 1u;
+        if (S.form == kPaired && run_model && S.shift == 0 && S.base == 0u) {
+            // a low-dose stream: zeros over the range, then its run events (jump
+            // the zero-bit (0,0) steps, take the step at the slot reached) up to
+            // the last pair the range needs, storing the nonzero counts inside it
+            for (int sc = lo; sc < hi; ++sc)
+                dst[(sc - lo) * P] = 0;
+            const uint32_t rt_sa = static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + S.model * kStates));
+            const int j_end = (hi + 1) >> 1;        // pairs [0, j_end) hold the range's scans
+            int j = 0;
+            while (j < j_end) {
+                const uint32_t t = tab_load(S.x, rt_sa);
+                j += static_cast<int>((t >> 14) & 63u);
+                if (j >= j_end)
+                    break;
+                if (S.bt.n < 10)
+                    S.bt.refill();
+                S.x = (t & 1023u) | S.bt.get(static_cast<int>((t >> 10) & 15u));
+                const uint32_t a = (t >> 20) & 15u, c = (t >> 24) & 15u;
+                if (a && 2 * j >= lo && 2 * j < hi)
+                    dst[(2 * j - lo) * P] = static_cast<T>(a);
+                if (c && 2 * j + 1 >= lo && 2 * j + 1 < hi)
+                    dst[(2 * j + 1 - lo) * P] = static_cast<T>(c);
+                ++j;
+            }
+            if (S.bt.consumed() > 8ll * S.tans_len)
+                report(st, kErrLength);
+        } else if (S.form == kPaired && S.two && S.shift == 0 && S.base == 0u) {
+            // a two-state stream without base or raw bits (models 8-31, tables in
+            // shared memory): the interleaved table steps up to the range's end
+            const uint32_t dec_sa = static_cast<uint32_t>(__cvta_generic_to_shared(s_dec + S.model * kStates));
+            const int last_seg = (hi - 1) >> 5;
+            for (int seg = 0; seg <= last_seg; ++seg) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; jj += 2) {
+                    const uint32_t ea = tab_load(S.x, dec_sa);
+                    const uint32_t eb = tab_load(S.x2, dec_sa);
+                    if (jj % 3 == 0 && S.bt.n < 30)
+                        S.bt.refill();
+                    pk[jj] = consume(ea, S.x, S.bt.lo, S.bt.hi, S.bt.n);
+                    if ((jj + 1) % 3 == 0 && S.bt.n < 30)
+                        S.bt.refill();
+                    pk[jj + 1] = consume(eb, S.x2, S.bt.lo, S.bt.hi, S.bt.n);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int sc = seg * 32 + i;
+                    if (sc >= lo && sc < hi)
+                        dst[(sc - lo) * P] = static_cast<T>((i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xFFFFu));
+                }
+            }
+            if (S.bt.consumed() > 8ll * S.tans_len)
+                report(st, kErrLength);
+        } else if (S.form == kPaired) {
+            // the run-decoded models' decode tables stay in global memory
+            const uint32_t *dec = (run_model ? dec_g : s_dec) + S.model * kStates;
             uint32_t over = 0;
             const int last_seg = (hi - 1) >> 5;
             for (int seg = 0; seg <= last_seg; ++seg) {
@@ -2989,6 +3045,7 @@ cudaError_t launch_decode_blocks(View v, Tables tb, long long first, long long n
 cudaError_t launch_decode_range(View v, Tables tb, long long first, long long n, void *out, DevStatus *status,
                                 cudaStream_t st)
 {
+    const int skip_count = __builtin_popcount(tb.skip_models);
     const size_t smem = kTableBytes;
     const cudaError_t e = v.w == 1 ? ensure_smem(reinterpret_cast<const void *>(k_decode_range<1>), smem)
                                    : ensure_smem(reinterpret_cast<const void *>(k_decode_range<2>), smem);
@@ -2998,9 +3055,11 @@ cudaError_t launch_decode_range(View v, Tables tb, long long first, long long n,
     long long grid = (blocks * v.P + 255) / 256;
     grid = grid < 1 ? 1 : (grid > 4ll * sm_count() ? 4ll * sm_count() : grid);
     if (v.w == 1)
-        k_decode_range<1><<<static_cast<int>(grid), 256, smem, st>>>(v, tb.dec, first, n, out, status);
+        k_decode_range<1><<<static_cast<int>(grid), 256, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                                                                      first, n, out, status);
     else
-        k_decode_range<2><<<static_cast<int>(grid), 256, smem, st>>>(v, tb.dec, first, n, out, status);
+        k_decode_range<2><<<static_cast<int>(grid), 256, smem, st>>>(v, tb.dec, tb.runs, tb.skip_models, skip_count,
+                                                                      first, n, out, status);
     return cudaGetLastError();
 }
 
