@@ -500,6 +500,10 @@ def run_profile_case(dev, torch, V, config="c4"):
     # launch 14: bright field with the index dropped (every disk pixel decoded pair by pair)
     res.drop_index()
     res.masked_sum(bf, out=out)
+    # one centre-of-mass moment query over the bright field (k_moments)
+    rr, cc = np.divmod(np.arange(w.n_pixels), w.det_cols)
+    wts = torch.from_numpy(np.stack([rr - w.det_rows // 2, cc - w.det_cols // 2]).astype(np.int32)).to(dev)
+    res.masked_moments(bf, wts)
     p = res.profile_read()
     print(json.dumps({"encode_s": t_enc, "kernels": p}), flush=True)
     res.free()
